@@ -1,0 +1,261 @@
+"""CPU oracle for Doge's Dynamic Mask Attention (DMA) hot path.
+
+TEST INFRASTRUCTURE ONLY.  Only the test-suite, the package smoke check and the
+benchmark's CPU-baseline leg may import this module.  The product path (the
+CUDA library and its Python binding) never calls it, and this module imports
+nothing from the product package.
+
+Everything here is a plain, slow, obviously-correct restatement of what the
+pages define, computed in numpy float64 (except where noted: the per-key score
+is handed on as float32, which is the precision the kernels and the dynamic
+mask use).  There is no blocking, fusion or reordering beyond what the
+definitions state.
+
+Source cited throughout (the only page that defines DMA):
+  "Transformers 中的 Doge 小语言模型完全指南：动态掩码注意力（DMA）与跨域 MoE（CDMoE）
+   架构解析与实战" (blog.gitcode.com), written below as [Guide].
+  [Guide §DMA.3]  section "动态掩码注意力（DMA）：从缓存 value states 生成稀疏掩码",
+                  forward chain step 3 (dt_proj, exp(A*softplus), prepare_dynamic_mask,
+                  top-k + scatter above keep_window_size).
+  [Guide §DMA.4]  same section, step 4 (scores scaled by head_dim**-0.5, fp32 softmax,
+                  additive attn_mask).
+  [Guide §DMA.init] same section, closing paragraph (A initialised with zeros).
+  [Guide §Config] section "DogeConfig 全参数详解" (num_key_value_heads, attention_bias=False,
+                  keep_window_size=2048, sliding_window=None -> full causal mask).
+
+Readings taken where the pages are silent (each one is listed with its reason in
+the design notes of the repository):
+  * dt_proj input is the per-token value row flattened head-major
+    (index h'*d + e) and projected to H_kv outputs; no bias (attention_bias=False).
+  * causal and padding masking are merged into the mask BEFORE the top-k, so a
+    row keeps the keep_window_size best keys among the keys it may see.
+  * ties in the top-k go to the lower key index.
+  * "exceeds keep_window_size" is strict: Lk > w triggers the top-k.
+  * the dt bias is added after scaling: s = scale * q.k + dt.
+  * GQA: query head h reads kv head g = h // (H_q / H_kv).
+  * min_dtype is bf16's lowest finite value.
+  * padded query rows (i >= len_b) are computed with the same formula.
+  * the decode query sits at position len_b - 1 and the cache holds it.
+
+Parity status of each function (pins live in tests/test_oracle_pins.py):
+  softplus, dt_scores            pinned (closed forms, worked example, flatten-order probe)
+  dynamic_mask_rows, kept_mask   pinned (brute-force rank count, closed forms, invariants,
+                                  torch.topk on tie-free rows)
+  thresholds                     pinned (rebuilds kept_mask exactly)
+  attention_rows, prefill        pinned (float64 SDPA, closed forms)
+  decode_step                    pinned (float64 SDPA, closed forms)
+"""
+from __future__ import annotations
+
+import numpy as np
+
+# bf16's lowest finite value, exactly representable in float32 and float64.
+MIN_DTYPE = -3.3895313892515355e38
+
+
+# --------------------------------------------------------------------------
+# S1: per-key score  dt = exp(A * softplus(dt_proj(value_states)))   [Guide §DMA.3]
+# --------------------------------------------------------------------------
+
+def softplus(x):
+    """softplus(x) = log(1 + exp(x)), written in the overflow-free form
+    max(x, 0) + log1p(exp(-|x|)) (same value, float64)."""
+    x = np.asarray(x, dtype=np.float64)
+    return np.maximum(x, 0.0) + np.log1p(np.exp(-np.abs(x)))
+
+
+def dt_scores64(v, W, A):
+    """Float64 per-key score [Guide §DMA.3].
+
+    v : [B, L, H_kv, d] value states (any float dtype; bf16 values pass exactly)
+    W : [H_kv*d, H_kv] dt_proj weight, input-major (x = v_flat @ W), no bias
+    A : [H_kv] one learnable scalar per kv head
+    returns dt64 [B, H_kv, L] float64
+    """
+    v = np.asarray(v, dtype=np.float64)
+    B, L, Hkv, d = v.shape
+    W = np.asarray(W, dtype=np.float64)
+    A = np.asarray(A, dtype=np.float64)
+    assert W.shape == (Hkv * d, Hkv) and A.shape == (Hkv,)
+    v_flat = v.reshape(B, L, Hkv * d)            # head-major: column h'*d + e
+    x = v_flat @ W                               # [B, L, H_kv]   dt_proj(value_states)
+    dt = np.exp(A[None, None, :] * softplus(x))  # exp(A * softplus(.))
+    return np.ascontiguousarray(dt.transpose(0, 2, 1))
+
+
+def dt_scores(v, W, A):
+    """dt rounded to float32, the precision the mask is built in: [B, H_kv, L]."""
+    return dt_scores64(v, W, A).astype(np.float32)
+
+
+# --------------------------------------------------------------------------
+# S2: dynamic mask   [Guide §DMA.3, prepare_dynamic_mask]
+# --------------------------------------------------------------------------
+
+def _valid_limit(row, len_b, Lq, Lk):
+    """Number of leading keys row `row` may see: causal (query position
+    row + Lk - Lq, so prefill row i sees keys <= i) and padding (keys >= len_b
+    are never seen).  For decode (Lq == 1) this is len_b: the query sits at
+    position len_b - 1 and sees every valid cached key."""
+    return min(row + (Lk - Lq) + 1, len_b)
+
+
+def dynamic_mask_rows(dt_row, len_b, Lq, Lk, w, rows):
+    """Additive mask rows for one (batch, kv head) [Guide §DMA.3].
+
+    dt_row : [Lk] float32 per-key score of this kv head
+    rows   : iterable of query rows
+    Each mask row starts as dt broadcast over the query rows; keys the row may
+    not see (causal or padding) are set to MIN_DTYPE; then, when Lk exceeds w,
+    only the w largest entries of the row are kept (ties: lower key index first,
+    a stable sort of the negated row) and every other entry becomes MIN_DTYPE.
+    returns float64 [len(rows), Lk]
+    """
+    dt_row = np.asarray(dt_row, dtype=np.float32).astype(np.float64)
+    rows = list(rows)
+    out = np.full((len(rows), Lk), MIN_DTYPE, dtype=np.float64)
+    for r, i in enumerate(rows):
+        lim = _valid_limit(i, len_b, Lq, Lk)
+        m = np.full(Lk, MIN_DTYPE, dtype=np.float64)
+        m[:lim] = dt_row[:lim]
+        if Lk > w:
+            order = np.argsort(-m, kind="stable")
+            keep = np.zeros(Lk, dtype=bool)
+            keep[order[:w]] = True
+            m[~keep] = MIN_DTYPE
+        out[r] = m
+    return out
+
+
+def kept_mask(dt, lengths, Lq, Lk, w):
+    """Boolean kept-key mask [B, H_kv, Lq, Lk] (small shapes only)."""
+    dt = np.asarray(dt, dtype=np.float32)
+    B, Hkv, _ = dt.shape
+    out = np.zeros((B, Hkv, Lq, Lk), dtype=bool)
+    for b in range(B):
+        for g in range(Hkv):
+            m = dynamic_mask_rows(dt[b, g], int(lengths[b]), Lq, Lk, w, range(Lq))
+            out[b, g] = m > MIN_DTYPE
+    return out
+
+
+def composite_key(dt_value, j):
+    """Total order used for the top-k: float32 bits of dt in the high word
+    (dt >= 0, so its bit pattern orders like the value), 0xFFFFFFFF - j in the
+    low word (so the lower index ranks higher on equal dt)."""
+    bits = int(np.asarray(dt_value, dtype=np.float32).view(np.uint32))
+    return (bits << 32) | (0xFFFFFFFF - int(j))
+
+
+def thresholds(dt, lengths, Lq, Lk, w):
+    """Row thresholds tau [B, H_kv, Lq] as uint64.
+
+    tau = composite key of the w-th best visible key when Lk > w and the row
+    sees more than w keys; else 0 (every visible key kept).  Key j is kept in a
+    row iff it is visible and composite_key(dt[j], j) >= tau.
+    """
+    dt = np.asarray(dt, dtype=np.float32)
+    B, Hkv, _ = dt.shape
+    tau = np.zeros((B, Hkv, Lq), dtype=np.uint64)
+    for b in range(B):
+        for g in range(Hkv):
+            for i in range(Lq):
+                lim = _valid_limit(i, int(lengths[b]), Lq, Lk)
+                if Lk > w and lim > w:
+                    order = np.argsort(-dt[b, g, :lim].astype(np.float64), kind="stable")
+                    j = int(order[w - 1])
+                    tau[b, g, i] = composite_key(dt[b, g, j], j)
+    return tau
+
+
+# --------------------------------------------------------------------------
+# S3: attention with the additive mask   [Guide §DMA.4]
+# --------------------------------------------------------------------------
+
+def attention_rows(q_rows, K, V, mask_rows, scale):
+    """softmax(scale * q K^T + mask) V for a block of query rows, float64.
+
+    q_rows [n, d], K [Lk, d], V [Lk, d], mask_rows [n, Lk] -> [n, d]
+    """
+    q_rows = np.asarray(q_rows, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    s = scale * (q_rows @ K.T) + mask_rows
+    s = s - s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    p = p / p.sum(axis=1, keepdims=True)
+    return p @ V
+
+
+def prefill_rows(q, k, v, dt, lengths, w, scale, b, h, rows):
+    """Output rows of one (batch b, query head h) of the prefill path.
+
+    q [B, L, H_q, d], k/v [B, L, H_kv, d], dt [B, H_kv, L] float32.
+    """
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    g = h // (Hq // Hkv)                                   # GQA group [Guide §Config]
+    rows = list(rows)
+    M = dynamic_mask_rows(dt[b, g], int(lengths[b]), L, L, w, rows)
+    return attention_rows(np.asarray(q[b, rows, h, :], dtype=np.float64),
+                          k[b, :, g, :], v[b, :, g, :], M, scale)
+
+
+def prefill(q, k, v, W, A, lengths, w, scale, dt=None, row_block=1024):
+    """Whole prefill forward: dt (unless given) -> dynamic mask -> attention.
+
+    Returns float64 [B, L, H_q, d].  dt, when given, is float32 [B, H_kv, L].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if dt is None:
+        dt = dt_scores(v, W, A)
+    dt = np.asarray(dt, dtype=np.float32)
+    n_rep = Hq // Hkv
+    out = np.empty((B, L, Hq, d), dtype=np.float64)
+    for b in range(B):
+        for g in range(Hkv):
+            for r0 in range(0, L, row_block):
+                rows = range(r0, min(L, r0 + row_block))
+                M = dynamic_mask_rows(dt[b, g], int(lengths[b]), L, L, w, rows)
+                for r in range(n_rep):
+                    h = g * n_rep + r
+                    out[b, r0:r0 + len(rows), h, :] = attention_rows(
+                        q[b, r0:r0 + len(rows), h, :], k[b, :, g, :], v[b, :, g, :], M, scale)
+    return out
+
+
+# --------------------------------------------------------------------------
+# S4: one decode step over a KV cache   [Guide §DMA.3 last paragraph, §DMA.4]
+# --------------------------------------------------------------------------
+
+def decode_step(q, k_cache, v_cache, W, A, lengths, w, scale, dt=None, batches=None):
+    """One query per sequence against its cache.
+
+    q [B, H_q, d]; k_cache / v_cache [B, Lk, H_kv, d]; the query sits at
+    position len_b - 1 and the cache already holds it.  dt is computed over the
+    whole cached value states (all Lk positions; positions >= len_b are masked).
+    Returns float64 [len(batches), H_q, d] (all batches by default).
+    """
+    B, Hq, d = q.shape
+    Lk, Hkv = k_cache.shape[1], k_cache.shape[2]
+    n_rep = Hq // Hkv
+    batches = range(B) if batches is None else list(batches)
+    out = np.empty((len(batches), Hq, d), dtype=np.float64)
+    for ob, b in enumerate(batches):
+        vb = np.asarray(v_cache[b], dtype=np.float64)            # [Lk, H_kv, d]
+        kb = np.asarray(k_cache[b], dtype=np.float64)
+        if dt is None:
+            dtb = dt_scores(vb[None], W, A)[0]                   # [H_kv, Lk] float32
+        else:
+            dtb = np.asarray(dt[b], dtype=np.float32)
+        for g in range(Hkv):
+            M = dynamic_mask_rows(dtb[g], int(lengths[b]), 1, Lk, w, [0])
+            for r in range(n_rep):
+                h = g * n_rep + r
+                out[ob, h, :] = attention_rows(np.asarray(q[b, h][None, :], dtype=np.float64),
+                                               kb[:, g, :], vb[:, g, :], M, scale)[0]
+    return out

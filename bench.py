@@ -1,0 +1,419 @@
+"""Benchmark of the DMA hot path on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--quick]
+
+Headline (`value`): prefill TFLOP/s on the dense-equivalent workload
+(B=8, L=2048, Hq=8, Hkv=4, d=64, keep_window_size=2048), counting 4*d FLOPs
+per kept (query, key) pair per query head; a step is one dma_forward_prefill
+call (dt scores, dynamic-mask selection, attention).  The same line reports
+decode GB/s (B=64, cache 65536, Hq=16, Hkv=8, d=128, w=2048; algorithmic KV
+bytes) and TFLOP/s of the sparse-padded and long-context prefill workloads.
+
+Timing: CUDA events per step on the launching stream, L2 flushed (256 MiB
+write) between timed steps, W untimed warm-up steps, a barrier and a device
+synchronize on both sides of the timed region, max over ranks.  Multi-GPU:
+one process per GPU (torchrun), every rank runs its own copy of the workload
+(weak scaling, no data-path collective).
+
+--impl reference times the CPU oracle (the only reference implementation of
+this method) on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from doge_dynamic_mask_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "DMA prefill TFLOP/s (kept keys) & decode KV GB/s, % of B200 peak"
+HEADLINE = "dense_eq"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------------------
+# work accounting (from the workload definition and the valid lengths)
+# ----------------------------------------------------------------------------
+
+def kept_pairs(L, w, lengths):
+    """Kept (query row, key) pairs per query head, summed over the batch: row i
+    of a sequence of valid length n keeps min(w, min(i+1, n)) keys when L > w,
+    else min(i+1, n)."""
+    total = 0
+    i = np.arange(L, dtype=np.int64)
+    for n in np.asarray(lengths, dtype=np.int64):
+        vis = np.minimum(i + 1, n)
+        total += int(np.minimum(vis, w).sum()) if L > w else int(vis.sum())
+    return total
+
+
+def prefill_flops(wl, lengths):
+    return 4 * wl.d * wl.Hq * kept_pairs(wl.L, wl.w, lengths)
+
+
+def decode_bytes(wl, lengths):
+    """V read for dt over the whole cache + the kept K and V rows + q and out."""
+    B, Lk, Hkv, d, Hq = wl.B, wl.L, wl.Hkv, wl.d, wl.Hq
+    v_scan = B * Lk * Hkv * d * 2
+    kept = sum(min(wl.w, int(n)) if Lk > wl.w else int(n) for n in lengths)
+    kv_rows = kept * Hkv * 2 * d * 2
+    return v_scan + kv_rows + 2 * B * Hq * d * 2
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region."""
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index),
+                 "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 7 and parts[0].isdigit():
+                    rows.append(parts)
+        except Exception:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [int(r[0]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[3 + k].lower() == "active"})
+        return {"sm_mhz": int(statistics.median(sm)), "sm_max_mhz": int(rows[0][1]), "reasons": reasons,
+                "samples": len(rows)}
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+def time_prefill(dma, wl, steps, warmup, flush, dev, ranks_sync):
+    x = make_inputs(wl, device=dev)
+    lengths = x["lengths"].cpu().numpy()
+    ws = dma.new_workspace(dma.dma_workspace_size(wl.B, wl.L, wl.L, wl.Hq, wl.Hkv, wl.d, wl.w), dev)
+    out = torch.empty_like(x["q"])
+
+    def step():
+        dma.dma_forward_prefill(x["q"], x["k"], x["v"], x["W"], x["A"], x["lengths"], wl.w, out=out, workspace=ws)
+
+    for _ in range(warmup):
+        step()
+        flush.zero_()
+    assert dma.dma_check(ws) == 0
+    ev = dma.StageEvents()
+    total_ms, stage = 0.0, [0.0, 0.0, 0.0]
+    ranks_sync()
+    with ev:
+        for _ in range(steps):
+            step()
+            torch.cuda.synchronize()
+            s1, s2, s3 = ev.stage_ms()
+            total_ms += s1 + s2 + s3
+            stage = [stage[0] + s1, stage[1] + s2, stage[2] + s3]
+            flush.zero_()
+    ranks_sync()
+    assert dma.dma_check(ws) == 0
+    flops = prefill_flops(wl, lengths)
+    return {"flops": flops, "ms": total_ms / steps, "stage_ms": [s / steps for s in stage], "launches": 3 * steps,
+            "x": x, "ws": ws, "out": out}
+
+
+def time_decode(dma, wl, steps, warmup, flush, dev, ranks_sync):
+    x = make_inputs(wl, device=dev)
+    lengths = x["lengths"].cpu().numpy()
+    ws = dma.new_workspace(dma.dma_workspace_size(wl.B, 1, wl.L, wl.Hq, wl.Hkv, wl.d, wl.w), dev)
+    out = torch.empty_like(x["q"])
+
+    def step():
+        dma.dma_decode_step(x["q"], x["k"], x["v"], x["W"], x["A"], x["lengths"], wl.w, out=out, workspace=ws)
+
+    for _ in range(warmup):
+        step()
+        flush.zero_()
+    assert dma.dma_check(ws) == 0
+    ev = dma.StageEvents()
+    total_ms, stage = 0.0, [0.0, 0.0, 0.0]
+    ranks_sync()
+    with ev:
+        for _ in range(steps):
+            step()
+            torch.cuda.synchronize()
+            s1, s2, s3 = ev.stage_ms()
+            total_ms += s1 + s2 + s3
+            stage = [stage[0] + s1, stage[1] + s2, stage[2] + s3]
+            flush.zero_()
+    ranks_sync()
+    assert dma.dma_check(ws) == 0
+    nbytes = decode_bytes(wl, lengths)
+    del x
+    return {"bytes": nbytes, "ms": total_ms / steps, "stage_ms": [s / steps for s in stage],
+            "launches": 4 * steps}
+
+
+def time_e2e(dma, wl, steps, warmup, dev):
+    """Same metric through the public call with host (pinned) buffers: the H2D
+    copy of every input and the D2H read of the output are inside each step."""
+    xh = {k: v.pin_memory() for k, v in make_inputs(wl, device="cpu").items()}
+    lengths = xh["lengths"].numpy()
+    xd = {k: torch.empty_like(v, device=dev) for k, v in xh.items()}
+    ws = dma.new_workspace(dma.dma_workspace_size(wl.B, wl.L, wl.L, wl.Hq, wl.Hkv, wl.d, wl.w), dev)
+    out_d = torch.empty_like(xd["q"])
+    out_h = torch.empty_like(xh["q"]).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in xh.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def step():
+        for k in xh:
+            xd[k].copy_(xh[k], non_blocking=True)
+        dma.dma_forward_prefill(xd["q"], xd["k"], xd["v"], xd["W"], xd["A"], xd["lengths"], wl.w, out=out_d,
+                                workspace=ws)
+        out_h.copy_(out_d, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return {"tflops": prefill_flops(wl, lengths) / (ms * 1e-3) / 1e12, "ms": ms, "h2d": h2d, "d2h": d2h}
+
+
+def cpu_baseline_prefill(wl, x, budget_s=12.0):
+    """The oracle as it stands on the host cores, on a bounded sample of rows of
+    the same workload: whole row blocks of batch 0, query head 0."""
+    import oracle
+    q = x["q"][0:1].float().cpu().numpy().astype(np.float64)
+    k = x["k"][0:1].float().cpu().numpy().astype(np.float64)
+    v = x["v"][0:1].float().cpu().numpy().astype(np.float64)
+    W = x["W"].double().cpu().numpy()
+    A = x["A"].double().cpu().numpy()
+    lengths = x["lengths"][0:1].cpu().numpy()
+    t0 = time.perf_counter()
+    dt = oracle.dt_scores(v, W, A)
+    rows_done, flops, block = 0, 0, 64
+    n_row = lengths[0]
+    while rows_done < wl.L and time.perf_counter() - t0 < budget_s:
+        rows = range(rows_done, min(wl.L, rows_done + block))
+        oracle.prefill_rows(q, k, v, dt, lengths, wl.w, wl.scale, 0, 0, rows)
+        for i in rows:
+            vis = min(i + 1, int(n_row))
+            flops += 4 * wl.d * (min(vis, wl.w) if wl.L > wl.w else vis)
+        rows_done += len(rows)
+    dt_s = time.perf_counter() - t0
+    return {"value": flops / dt_s / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"{wl.name}: batch 0, query head 0, rows 0..{rows_done - 1} of {wl.L} "
+                      f"(dt of the whole sequence included), {dt_s:.1f} s"}
+
+
+def run_ours(args):
+    from doge_dynamic_mask_b200 import dma
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        pg = dist
+
+    def ranks_sync():
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v):
+        if pg is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks = load_peaks()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    wl = WORKLOADS[HEADLINE]
+    with ClockSampler(local) as clk:
+        head = time_prefill(dma, wl, args.steps, args.warmup, flush, dev, ranks_sync)
+    clocks = clk.summary()
+    ms = max_over_ranks(head["ms"])
+    att_ms = max_over_ranks(head["stage_ms"][2])
+    value = world * head["flops"] / (ms * 1e-3) / 1e12
+    att_tflops = head["flops"] / (att_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "attn_prefill_kernel<64>", "achieved": round(att_tflops, 2),
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(att_tflops / peaks["bf16_tflops"], 4),
+                "peak_source": f"{peaks['source']} bf16 burst", "traffic": None,
+                "per_launch": {"flops": head["flops"], "ms": round(att_ms, 5)}}
+
+    result = {"metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+              "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+              "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+              "data": "synthetic",
+              "config": {"workload": wl.name, "B": wl.B, "L": wl.L, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d,
+                         "keep_window_size": wl.w, "l2": "flushed between timed steps (256 MiB write)",
+                         "parallelism": f"replicas{world}"},
+              "stage_ms": {"dt": round(head["stage_ms"][0], 5), "select": round(head["stage_ms"][1], 5),
+                           "attention": round(head["stage_ms"][2], 5)},
+              "roofline": roofline, "gpu_launches": head["launches"], "clocks": clocks}
+    del head
+
+    # the other workloads of the same method (same timing rules)
+    others = {}
+    if not args.quick:
+        for name in ("sparse_pad", "long"):
+            o = time_prefill(dma, WORKLOADS[name], args.steps, args.warmup, flush, dev, ranks_sync)
+            oms = max_over_ranks(o["ms"])
+            a_ms = max_over_ranks(o["stage_ms"][2])
+            others[name] = {"value": round(o["flops"] / (oms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                            "ms_per_step": round(oms, 5),
+                            "attention_tflops": round(o["flops"] / (a_ms * 1e-3) / 1e12, 2),
+                            "attention_frac": round(o["flops"] / (a_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+                            "stage_ms": [round(s, 5) for s in o["stage_ms"]]}
+            result["gpu_launches"] += o["launches"]
+            del o
+            torch.cuda.empty_cache()
+        d = time_decode(dma, WORKLOADS["decode"], args.steps, args.warmup, flush, dev, ranks_sync)
+        dms = max_over_ranks(d["ms"])
+        dt_ms = max_over_ranks(d["stage_ms"][0])
+        gbs = d["bytes"] / (dms * 1e-3) / 1e9
+        v_scan = WORKLOADS["decode"].B * WORKLOADS["decode"].L * WORKLOADS["decode"].Hkv * WORKLOADS["decode"].d * 2
+        others["decode"] = {"value": round(world * gbs, 1), "unit": "GB/s", "ms_per_step": round(dms, 5),
+                            "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                            "bytes_per_step": d["bytes"], "stage_ms": [round(s, 5) for s in d["stage_ms"]],
+                            "dt_kernel_gbs": round(v_scan / (dt_ms * 1e-3) / 1e9, 1)}
+        result["gpu_launches"] += d["launches"]
+        del d
+        torch.cuda.empty_cache()
+    result["workloads"] = others
+
+    e2e = time_e2e(dma, wl, max(3, args.steps), args.warmup, dev)
+    result["e2e"] = {"value": round(world * e2e["tflops"], 3), "unit": "TFLOP/s", "h2d_bytes_per_step": e2e["h2d"],
+                     "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": round(e2e["ms"], 4)}
+    if rank == 0:
+        x = make_inputs(wl, device="cpu")
+        result["cpu_baseline"] = cpu_baseline_prefill(wl, x)
+        print(json.dumps(result), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = WORKLOADS[HEADLINE]
+    x = make_inputs(wl, device="cpu")
+    lengths = x["lengths"].numpy()
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline_prefill(wl, x, budget_s=4.0)
+        if i >= args.warmup:
+            per_step.append(r)
+    value = statistics.mean(r["value"] for r in per_step)
+    total_flops = prefill_flops(wl, lengths)
+    line = {"metric": METRIC, "impl": "reference", "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_flops / (value * 1e12) * 1e3 if value > 0 else None,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "L": wl.L, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d,
+                       "keep_window_size": wl.w},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": per_step[0]["cores"], "kind": "oracle",
+                             "sample": per_step[0]["sample"] + " per step; ms_per_step extrapolated to the whole workload"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--quick", action="store_true", help="headline workload only")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,90 @@
+// Internal constants, workspace plan layouts and kernel launchers of libdma.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace dma {
+
+// Query rows per prefill row tile and keys per attention key tile.
+constexpr int kRowTile = 128;
+constexpr int kKeyTile = 128;
+// Keys per split of the decode attention.
+constexpr int kDecodeChunk = 128;
+// Largest keep_window_size the selectors accept when the top-k is active.
+constexpr int kMaxKeep = 8192;
+// Longest key axis (key indices live in 16..31 bits of the composite key and
+// the selectors count in 32-bit words).
+constexpr int kMaxLen = 1 << 20;
+// Bounded waits give up after this many SM clock cycles (about one second).
+constexpr long long kWaitLimitCycles = 2000000000LL;
+
+// Device-side error codes recorded in the workspace's status word.
+enum DeviceError : uint32_t {
+  kDevErrNone = 0,
+  kDevErrBadLength = 6,      // a lengths[b] outside [1, Lk]
+  kDevErrTimeoutBase = 100,  // 100 + site: a bounded wait gave up
+};
+
+// Workspace header: status word at offset 0; the rest of the first 256 bytes is reserved.
+constexpr size_t kHeaderBytes = 256;
+
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Per-(batch, kv head, row tile) compacted key list produced by the prefill
+// selector and consumed by the prefill attention kernel.
+//   idx [tiles][cap]  int32   key index j
+//   bias[tiles][cap]  float   dt[b, g, j]
+//   span[tiles][cap]  uint32  lo | hi << 16: the key is kept on tile rows [lo, hi)
+//   counts[tiles]     int2    (n_full, n_total); entries [0, n_full) are kept by
+//                             every row of the tile; entries past n_total up to
+//                             the next multiple of kKeyTile are padding (span 0).
+// tiles are ordered ((b * Hkv + g) * n_row_tiles + t).
+struct PrefillPlan {
+  float* dt;        // [B, Hkv, L]
+  uint64_t* tau;    // [B, Hkv, L] row thresholds
+  int32_t* idx;
+  float* bias;
+  uint32_t* span;
+  int2* counts;
+  int cap;          // entries per tile (multiple of kKeyTile)
+  int n_row_tiles;
+};
+
+// Decode plan: per (batch, kv head) the kept keys in ascending index order.
+struct DecodePlan {
+  float* dt;        // [B, Hkv, Lk]
+  uint64_t* tau;    // [B, Hkv]
+  int32_t* idx;     // [B, Hkv, cap]
+  float* bias;      // [B, Hkv, cap]
+  int32_t* count;   // [B, Hkv]
+  float* part;      // [B, Hq, n_split, d + 2]  (o[d], m, l)
+  int cap;          // multiple of kDecodeChunk
+  int n_split;
+};
+
+struct Geometry {
+  int B, Lq, Lk, Hq, Hkv, d, w;
+};
+
+size_t prefill_plan_bytes(const Geometry& g);
+size_t decode_plan_bytes(const Geometry& g);
+PrefillPlan carve_prefill_plan(void* ws, const Geometry& g);
+DecodePlan carve_decode_plan(void* ws, const Geometry& g);
+
+// launchers (return cudaGetLastError() after the launch)
+cudaError_t launch_dt_scores(const void* v, const float* W, const float* A, int B, int L, int Hkv, int d,
+                             float* dt, cudaStream_t s);
+cudaError_t launch_select_prefill(const float* dt, const int32_t* lengths, const Geometry& g,
+                                  const PrefillPlan& plan, uint32_t* err, cudaStream_t s);
+cudaError_t launch_select_decode(const float* dt, const int32_t* lengths, const Geometry& g,
+                                 const DecodePlan& plan, uint32_t* err, cudaStream_t s);
+cudaError_t launch_prefill_bitmask(const PrefillPlan& plan, const Geometry& g, uint32_t* bitmask, cudaStream_t s);
+cudaError_t launch_decode_bitmask(const DecodePlan& plan, const Geometry& g, uint32_t* bitmask, cudaStream_t s);
+cudaError_t launch_attn_prefill(const void* q, const void* k, const void* v, const Geometry& g, float scale,
+                                const PrefillPlan& plan, void* out, uint32_t* err, cudaStream_t s);
+cudaError_t launch_attn_decode(const void* q, const void* k, const void* v, const Geometry& g, float scale,
+                               const DecodePlan& plan, void* out, cudaStream_t s);
+
+}  // namespace dma

@@ -1,0 +1,321 @@
+// S2: the dynamic mask's causal top-k, as compact plans for the attention kernels.
+//
+// Method: page "Transformers 中的 Doge 小语言模型完全指南", section
+// "动态掩码注意力（DMA）：从缓存 value states 生成稀疏掩码", step 3
+// (prepare_dynamic_mask: dt broadcast over the query rows, padding set to
+// min_dtype, and above keep_window_size only the keep_window_size best
+// positions of each row survive).  Causal masking is merged before the top-k,
+// ties go to the lower key index.
+//
+// Prefill (one CTA per (batch, kv head, 128-row tile)).  dt does not depend on
+// the query, so the row threshold tau_i (the composite key of row i's worst
+// kept key) never decreases along the rows: each key is kept on one contiguous
+// interval of rows, and the union of the kept sets of a row tile is the w keys
+// kept at its first row plus at most 127 newer keys.  The CTA
+//   1. radix-selects tau at the tile's first row over the keys it sees,
+//   2. collects the union U (keys <= the tile's last visible row whose key is
+//      >= that tau) in index order,
+//   3. takes the 128 smallest keys of U, in which every later row's tau lies,
+//      and resolves tau_i for each row of the tile,
+//   4. gives each key of U its row interval [lo, hi) inside the tile and writes
+//      the list: keys kept by every row first, then the rest (index order in
+//      each class), each with its dt bias and interval.
+// Tiles whose rows see at most w keys (and every tile when Lk <= w) keep every
+// visible key and skip the selection.
+//
+// Decode (one CTA per (batch, kv head)): the single query at len_b - 1 keeps
+// the w best of its len_b keys; radix-select the w-th key, then compact the
+// kept keys in index order.
+#include "select_common.cuh"
+
+namespace dma {
+namespace {
+
+struct SelectSmem {
+  uint32_t hist[kBins];
+  uint64_t cand[kCandCap];
+  uint32_t red[64];
+  uint64_t vars[8];
+  uint64_t tau_s[kRowTile];
+  uint64_t bot[kRowTile];
+  uint64_t bot_raw[kRowTile];
+  int misc[8];
+  // followed by U[ucap] (uint64) in dynamic shared memory
+};
+
+__device__ __forceinline__ int clamp_len(const int32_t* lengths, int b, int L, uint32_t* err) {
+  int len = lengths ? lengths[b] : L;
+  if (len < 1 || len > L) {
+    if (threadIdx.x == 0) raise_error(err, kDevErrBadLength);
+    len = len < 1 ? 1 : L;
+  }
+  return len;
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_prefill_kernel(const float* __restrict__ dt,
+                                                                     const int32_t* __restrict__ lengths, int Hkv,
+                                                                     int L, int w, PrefillPlan plan,
+                                                                     uint32_t* err) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SelectSmem& sm = *reinterpret_cast<SelectSmem*>(smem_raw);
+  uint64_t* U = reinterpret_cast<uint64_t*>(smem_raw + sizeof(SelectSmem));
+  SelScratch sc{sm.hist, sm.cand, sm.red, sm.vars};
+
+  const int t = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int len = clamp_len(lengths, b, L, err);
+  const int r0 = t * kRowTile;
+  const int nrows = min(kRowTile, L - r0);
+  const int p = min(r0, len - 1);                 // effective position of the first row
+  const int q = min(r0 + nrows - 1, len - 1);     // effective position of the last row
+  const bool topk = L > w;
+  const size_t bg = static_cast<size_t>(b) * Hkv + g;
+  const uint32_t* bits = reinterpret_cast<const uint32_t*>(dt) + bg * L;
+  uint64_t* tau_g = plan.tau + bg * L;
+  const size_t tile = bg * plan.n_row_tiles + t;
+  int32_t* idx_o = plan.idx + tile * plan.cap;
+  float* bias_o = plan.bias + tile * plan.cap;
+  uint32_t* span_o = plan.span + tile * plan.cap;
+  const int tid = threadIdx.x;
+
+  if (!topk || q + 1 <= w) {
+    // every visible key of every row is kept: keys <= r0 by all rows, key j > r0 from row j on
+    const int n_full = min(r0, q) + 1;
+    const int n_total = q + 1;
+    for (int i = tid; i < nrows; i += blockDim.x) tau_g[r0 + i] = 0ull;
+    for (int j = tid; j < n_total; j += blockDim.x) {
+      idx_o[j] = j;
+      bias_o[j] = __uint_as_float(bits[j]);
+      const int lo = j > r0 ? j - r0 : 0;
+      span_o[j] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(nrows) << 16);
+    }
+    const int padded = (n_total + kKeyTile - 1) / kKeyTile * kKeyTile;
+    for (int j = n_total + tid; j < padded; j += blockDim.x) {
+      idx_o[j] = 0;
+      bias_o[j] = 0.0f;
+      span_o[j] = 0u;
+    }
+    if (tid == 0) plan.counts[tile] = make_int2(n_full, n_total);
+    return;
+  }
+
+  // 1. threshold at the first row
+  uint64_t tau0 = 0ull;
+  if (p + 1 > w) tau0 = select_kth_global(bits, p + 1, static_cast<uint32_t>(w), sc);
+  const int n_old = p + 1 > w ? w : p + 1;
+
+  // 2. the union U of kept keys, in index order
+  const int nU = ordered_compact(
+      q + 1, [&](int j) { return composite_key(bits[j], j) >= tau0; },
+      [&](int pos, int j) { U[pos] = composite_key(bits[j], j); }, sc);
+  __syncthreads();
+
+  // 3. the kRowTile smallest keys of U, ascending; then tau for every row
+  const int nbot = min(nU, kRowTile);
+  uint64_t sigma = ~0ull;
+  if (nU > kRowTile) sigma = select_kth_smem(U, nU, static_cast<uint32_t>(nU - kRowTile + 1), sc);
+  if (tid == 0) sm.misc[0] = 0;
+  __syncthreads();
+  for (int e = tid; e < nU; e += blockDim.x) {
+    if (U[e] <= sigma) {
+      const int pos = atomicAdd(&sm.misc[0], 1);
+      if (pos < kRowTile) sm.bot_raw[pos] = U[e];
+    }
+  }
+  __syncthreads();
+  if (tid < nbot) {
+    const uint64_t key = sm.bot_raw[tid];
+    int rank = 0;
+    for (int f = 0; f < nbot; ++f) rank += sm.bot_raw[f] < key;
+    sm.bot[rank] = key;
+  }
+  __syncthreads();
+  if (tid < kRowTile) {
+    uint64_t tau = ~0ull;   // rows past the end of the sequence axis: unused
+    if (tid < nrows) {
+      const int ip = min(r0 + tid, len - 1);
+      if (ip + 1 <= w) {
+        tau = 0ull;
+      } else {
+        // keys of U visible to this row: the n_old old keys plus new keys j <= ip
+        int lo = n_old, hi = nU;
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (static_cast<int>(composite_index(U[mid])) <= ip) lo = mid + 1; else hi = mid;
+        }
+        const int rank = lo - w + 1;   // ascending rank of the row's w-th best key
+        int c = 0;
+        tau = 0ull;
+        for (int e = 0; e < nbot; ++e) {
+          const uint64_t key = sm.bot[e];
+          if (static_cast<int>(composite_index(key)) <= ip && ++c == rank) {
+            tau = key;
+            break;
+          }
+        }
+      }
+      tau_g[r0 + tid] = tau;
+    }
+    sm.tau_s[tid] = tau;
+  }
+  __syncthreads();
+
+  // 4. row intervals and the two-class ordered list
+  const int per = (nU + blockDim.x - 1) / blockDim.x;
+  const int e0 = tid * per, e1 = min(nU, e0 + per);
+  uint32_t nf = 0, np = 0;
+  for (int e = e0; e < e1; ++e) {
+    const uint64_t key = U[e];
+    const int j = static_cast<int>(composite_index(key));
+    const int lo = j > r0 ? j - r0 : 0;
+    int a = 0, c = nrows;   // first row whose tau exceeds the key
+    while (a < c) {
+      const int mid = (a + c) >> 1;
+      if (sm.tau_s[mid] > key) c = mid; else a = mid + 1;
+    }
+    const int hi = a;
+    if (hi > lo) {
+      if (lo == 0 && hi == nrows) ++nf; else ++np;
+    }
+  }
+  uint32_t total;
+  const uint32_t base = block_exclusive_scan(nf | (np << 16), sm.red, &total);
+  const int n_full = static_cast<int>(total & 0xFFFFu);
+  const int n_total = n_full + static_cast<int>(total >> 16);
+  uint32_t pf = base & 0xFFFFu, pp = n_full + (base >> 16);
+  for (int e = e0; e < e1; ++e) {
+    const uint64_t key = U[e];
+    const int j = static_cast<int>(composite_index(key));
+    const int lo = j > r0 ? j - r0 : 0;
+    int a = 0, c = nrows;
+    while (a < c) {
+      const int mid = (a + c) >> 1;
+      if (sm.tau_s[mid] > key) c = mid; else a = mid + 1;
+    }
+    const int hi = a;
+    if (hi > lo) {
+      const uint32_t pos = (lo == 0 && hi == nrows) ? pf++ : pp++;
+      idx_o[pos] = j;
+      bias_o[pos] = __uint_as_float(static_cast<uint32_t>(key >> 32));
+      span_o[pos] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+    }
+  }
+  const int padded = (n_total + kKeyTile - 1) / kKeyTile * kKeyTile;
+  for (int j = n_total + tid; j < padded; j += blockDim.x) {
+    idx_o[j] = 0;
+    bias_o[j] = 0.0f;
+    span_o[j] = 0u;
+  }
+  if (tid == 0) plan.counts[tile] = make_int2(n_full, n_total);
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_decode_kernel(const float* __restrict__ dt,
+                                                                    const int32_t* __restrict__ lengths, int Hkv,
+                                                                    int Lk, int w, DecodePlan plan, uint32_t* err) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SelectSmem& sm = *reinterpret_cast<SelectSmem*>(smem_raw);
+  SelScratch sc{sm.hist, sm.cand, sm.red, sm.vars};
+  const int g = blockIdx.x, b = blockIdx.y;
+  const int len = clamp_len(lengths, b, Lk, err);
+  const size_t bg = static_cast<size_t>(b) * Hkv + g;
+  const uint32_t* bits = reinterpret_cast<const uint32_t*>(dt) + bg * Lk;
+  int32_t* idx_o = plan.idx + bg * plan.cap;
+  float* bias_o = plan.bias + bg * plan.cap;
+  const int tid = threadIdx.x;
+  int n;
+  uint64_t tau = 0ull;
+  if (Lk > w && len > w) {
+    tau = select_kth_global(bits, len, static_cast<uint32_t>(w), sc);
+    n = ordered_compact(
+        len, [&](int j) { return composite_key(bits[j], j) >= tau; },
+        [&](int pos, int j) {
+          idx_o[pos] = j;
+          bias_o[pos] = __uint_as_float(bits[j]);
+        },
+        sc);
+  } else {
+    n = len;
+    for (int j = tid; j < len; j += blockDim.x) {
+      idx_o[j] = j;
+      bias_o[j] = __uint_as_float(bits[j]);
+    }
+  }
+  const int padded = (n + kDecodeChunk - 1) / kDecodeChunk * kDecodeChunk;
+  for (int j = n + tid; j < padded; j += blockDim.x) {
+    idx_o[j] = 0;
+    bias_o[j] = 0.0f;
+  }
+  if (tid == 0) {
+    plan.count[bg] = n;
+    plan.tau[bg] = tau;
+  }
+}
+
+// Dense bitmask [B, Hkv, L, ceil(L/32)] from the prefill plan (tests/debug).
+__global__ void prefill_bitmask_kernel(PrefillPlan plan, int Hkv, int L, uint32_t* bm) {
+  const int t = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const size_t bg = static_cast<size_t>(b) * Hkv + g;
+  const size_t tile = bg * plan.n_row_tiles + t;
+  const int words = (L + 31) / 32;
+  const int2 cnt = plan.counts[tile];
+  const int r0 = t * kRowTile;
+  for (int e = threadIdx.x; e < cnt.y; e += blockDim.x) {
+    const int j = plan.idx[tile * plan.cap + e];
+    const uint32_t sp = plan.span[tile * plan.cap + e];
+    const int lo = sp & 0xFFFF, hi = sp >> 16;
+    for (int r = lo; r < hi; ++r)
+      atomicOr(&bm[(bg * L + r0 + r) * words + (j >> 5)], 1u << (j & 31));
+  }
+}
+
+__global__ void decode_bitmask_kernel(DecodePlan plan, int Hkv, int Lk, uint32_t* bm) {
+  const int g = blockIdx.x, b = blockIdx.y;
+  const size_t bg = static_cast<size_t>(b) * Hkv + g;
+  const int words = (Lk + 31) / 32;
+  const int n = plan.count[bg];
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    const int j = plan.idx[bg * plan.cap + e];
+    atomicOr(&bm[bg * words + (j >> 5)], 1u << (j & 31));
+  }
+}
+
+size_t select_smem_bytes(int ucap) { return sizeof(SelectSmem) + static_cast<size_t>(ucap) * sizeof(uint64_t); }
+
+}  // namespace
+
+cudaError_t launch_select_prefill(const float* dt, const int32_t* lengths, const Geometry& g,
+                                  const PrefillPlan& plan, uint32_t* err, cudaStream_t s) {
+  const int L = g.Lk;
+  const int ucap = L > g.w ? g.w + kRowTile : 0;
+  const size_t smem = select_smem_bytes(ucap);
+  cudaError_t e = cudaFuncSetAttribute(select_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(plan.n_row_tiles, g.Hkv, g.B);
+  select_prefill_kernel<<<grid, kSelThreads, smem, s>>>(dt, lengths, g.Hkv, L, g.w, plan, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_decode(const float* dt, const int32_t* lengths, const Geometry& g,
+                                 const DecodePlan& plan, uint32_t* err, cudaStream_t s) {
+  const size_t smem = select_smem_bytes(0);
+  cudaError_t e = cudaFuncSetAttribute(select_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(g.Hkv, g.B);
+  select_decode_kernel<<<grid, kSelThreads, smem, s>>>(dt, lengths, g.Hkv, g.Lk, g.w, plan, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_bitmask(const PrefillPlan& plan, const Geometry& g, uint32_t* bitmask, cudaStream_t s) {
+  dim3 grid(plan.n_row_tiles, g.Hkv, g.B);
+  prefill_bitmask_kernel<<<grid, 256, 0, s>>>(plan, g.Hkv, g.Lk, bitmask);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_bitmask(const DecodePlan& plan, const Geometry& g, uint32_t* bitmask, cudaStream_t s) {
+  dim3 grid(g.Hkv, g.B);
+  decode_bitmask_kernel<<<grid, 256, 0, s>>>(plan, g.Hkv, g.Lk, bitmask);
+  return cudaGetLastError();
+}
+
+}  // namespace dma

@@ -1,0 +1,176 @@
+"""Thin Python binding of libdma (argument marshalling only).
+
+Every function here forwards to the C entry point of the same name in
+``libdma.so`` (declared in include/dma.h) with device pointers taken from torch
+tensors and the current torch CUDA stream.  No step of the computation runs in
+Python, and there is no fallback: importing this module fails loudly if the
+library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdma.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"libdma.so is not built ({_LIB_PATH}); run `python -m doge_dynamic_mask_b200.build` (needs nvcc)")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+DMA_OK = 0
+STATUS = {0: "DMA_OK", 1: "DMA_ERR_INVALID_ARG", 2: "DMA_ERR_UNSUPPORTED", 3: "DMA_ERR_WORKSPACE",
+          4: "DMA_ERR_CUDA", 5: "DMA_ERR_TIMEOUT", 6: "DMA_ERR_BAD_LENGTH"}
+
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_lib.dma_workspace_size.restype = _sz
+_lib.dma_workspace_size.argtypes = [_i] * 7
+_lib.dma_dt_scores.restype = _i
+_lib.dma_dt_scores.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp]
+_lib.dma_build_mask.restype = _i
+_lib.dma_build_mask.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]
+_lib.dma_forward_prefill.restype = _i
+_lib.dma_forward_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _sz,
+                                     _vp]
+_lib.dma_decode_step.restype = _i
+_lib.dma_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _sz, _vp]
+_lib.dma_check.restype = _i
+_lib.dma_check.argtypes = [_vp, _i, _vp]
+_lib.dma_status_string.restype = ctypes.c_char_p
+_lib.dma_status_string.argtypes = [_i]
+_lib.dma_last_cuda_error.restype = _i
+_lib.dma_last_cuda_error.argtypes = []
+_lib.dma_set_stage_events.restype = _i
+_lib.dma_set_stage_events.argtypes = [_vp, _i]
+
+
+class DMAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        name = _lib.dma_status_string(status).decode()
+        extra = f" (cudaError {_lib.dma_last_cuda_error()})" if status == 4 else ""
+        super().__init__(f"{where}: {name}{extra}")
+        self.status = status
+
+
+def _ok(status: int, where: str):
+    if status != DMA_OK:
+        raise DMAError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libdma must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def dma_workspace_size(B, Lq, Lk, Hq, Hkv, d, keep_window_size) -> int:
+    return int(_lib.dma_workspace_size(B, Lq, Lk, Hq, Hkv, d, keep_window_size))
+
+
+def new_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A zeroed device workspace (the status word must start at zero)."""
+    return torch.zeros(int(nbytes), dtype=torch.uint8, device=device or "cuda")
+
+
+def dma_dt_scores(v, W_dt, A, dt_out=None, stream=None):
+    B, L, Hkv, d = v.shape
+    if dt_out is None:
+        dt_out = torch.empty((B, Hkv, L), dtype=torch.float32, device=v.device)
+    _ok(_lib.dma_dt_scores(_ptr(v), _ptr(W_dt), _ptr(A), B, L, Hkv, d, _ptr(dt_out), _stream(stream)),
+        "dma_dt_scores")
+    return dt_out
+
+
+def dma_build_mask(dt, lengths, Lq, keep_window_size, workspace=None, tau_out=None, bitmask_out=None,
+                   stream=None):
+    B, Hkv, Lk = dt.shape
+    if workspace is None:
+        workspace = new_workspace(dma_workspace_size(B, Lq, Lk, Hkv, Hkv, 64, keep_window_size), dt.device)
+    _ok(_lib.dma_build_mask(_ptr(dt), _ptr(lengths), B, Hkv, Lq, Lk, keep_window_size, _ptr(tau_out),
+                            _ptr(bitmask_out), _ptr(workspace), workspace.numel(), _stream(stream)),
+        "dma_build_mask")
+    return workspace
+
+
+def dma_forward_prefill(q, k, v, W_dt, A, lengths, keep_window_size, scale=None, dt_in=None, out=None,
+                        workspace=None, stream=None):
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = new_workspace(dma_workspace_size(B, L, L, Hq, Hkv, d, keep_window_size), q.device)
+    _ok(_lib.dma_forward_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(W_dt), _ptr(A), _ptr(lengths), B, L, Hq, Hkv, d,
+                                 keep_window_size, float(scale), _ptr(dt_in), _ptr(out), _ptr(workspace),
+                                 workspace.numel(), _stream(stream)),
+        "dma_forward_prefill")
+    return out
+
+
+def dma_decode_step(q, k_cache, v_cache, W_dt, A, lengths, keep_window_size, scale=None, dt_in=None, out=None,
+                    workspace=None, stream=None):
+    B, Hq, d = q.shape
+    Lk, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = new_workspace(dma_workspace_size(B, 1, Lk, Hq, Hkv, d, keep_window_size), q.device)
+    _ok(_lib.dma_decode_step(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(W_dt), _ptr(A), _ptr(lengths), B, Lk, Hq,
+                             Hkv, d, keep_window_size, float(scale), _ptr(dt_in), _ptr(out), _ptr(workspace),
+                             workspace.numel(), _stream(stream)),
+        "dma_decode_step")
+    return out
+
+
+def dma_check(workspace, clear=True, stream=None) -> int:
+    """Synchronises the stream and returns the device-recorded status (0 = DMA_OK)."""
+    return int(_lib.dma_check(_ptr(workspace), 1 if clear else 0, _stream(stream)))
+
+
+class StageEvents:
+    """Context manager: while active, prefill/decode calls on this thread record
+    4 torch CUDA events (before S1, after S1, after S2, after the attention)."""
+
+    def __init__(self):
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        for e in self.events:          # materialise the underlying cudaEvent_t
+            e.record()
+        self._arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in self.events])
+
+    def __enter__(self):
+        _ok(_lib.dma_set_stage_events(self._arr, 4), "dma_set_stage_events")
+        return self
+
+    def __exit__(self, *exc):
+        _lib.dma_set_stage_events(None, 0)
+
+    def stage_ms(self):
+        """(S1, S2, attention) milliseconds of the last recorded call."""
+        e = self.events
+        return (e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3]))
+
+
+def dma_status_string(status: int) -> str:
+    return _lib.dma_status_string(status).decode()
+
+
+def raw():
+    """The ctypes handle (for tests that call the C ABI with raw pointers)."""
+    return _lib

@@ -1,0 +1,157 @@
+/*
+ * libdma — C ABI of the B200 (sm_100a) hot path of Doge's Dynamic Mask Attention.
+ *
+ * Source of the method: the page "Transformers 中的 Doge 小语言模型完全指南：
+ * 动态掩码注意力（DMA）与跨域 MoE（CDMoE）架构解析与实战" (blog.gitcode.com), section
+ * "动态掩码注意力（DMA）：从缓存 value states 生成稀疏掩码" (written [DMA] below; its
+ * forward-chain steps are [DMA step 3] and [DMA step 4]) and section
+ * "DogeConfig 全参数详解" ([Config]).
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or retains them, and keeps no per-call state.
+ *   - bf16 tensors are passed as `const void*` and hold IEEE bfloat16 values.
+ *   - Layouts are dense row-major, innermost dimension last:
+ *       q (prefill)   [B, L, Hq, d]        q (decode) [B, Hq, d]
+ *       k, v          [B, L, Hkv, d]       caches     [B, Lk, Hkv, d]
+ *       out           same layout as q
+ *       W_dt          [Hkv*d, Hkv] float32, input-major: x[g] = sum_c v_flat[c] * W_dt[c, g],
+ *                     with v_flat[h'*d + e] = v[h', e] (head-major flattening); no bias
+ *       A             [Hkv] float32
+ *       dt            [B, Hkv, L] float32
+ *       lengths       [B] int32 valid lengths (right padding), or NULL = all full
+ *   - GQA: query head h reads kv head g = h / (Hq / Hkv).
+ *   - Every pointer must be 16-byte aligned.  Supported: d in {64, 128},
+ *     Hkv in {1, 2, 4, 8, 16}, Hq a multiple of Hkv with Hq/Hkv <= 8,
+ *     L (or Lk) in [1, 2^20], keep_window_size >= 1 (at most 8192 whenever
+ *     the key length exceeds it), an sm_100 device.
+ *   - Calls are asynchronous on `stream` and return a status at once; they only
+ *     fail synchronously on argument errors and launch errors.  Faults found
+ *     on the device (a length outside [1, Lk], a bounded wait that gave up) are
+ *     recorded in the workspace's status word; read them with dma_check().
+ *   - A workspace must be zeroed once before its first use (the status word
+ *     lives in its first bytes); kernels only ever set that word.
+ *   - Calls on different streams must use different workspaces.
+ */
+#ifndef DMA_H_
+#define DMA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define DMA_API __attribute__((visibility("default")))
+#else
+#define DMA_API
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* dma_stream_t;
+
+typedef enum {
+  DMA_OK = 0,
+  DMA_ERR_INVALID_ARG = 1, /* NULL pointer, non-positive size, Hq % Hkv != 0, misaligned pointer */
+  DMA_ERR_UNSUPPORTED = 2, /* shape outside the supported set, or not an sm_100 device */
+  DMA_ERR_WORKSPACE = 3,   /* workspace smaller than dma_workspace_size() */
+  DMA_ERR_CUDA = 4,        /* a CUDA call failed; dma_last_cuda_error() has the code */
+  DMA_ERR_TIMEOUT = 5,     /* a bounded device wait gave up (reported by dma_check) */
+  DMA_ERR_BAD_LENGTH = 6   /* a lengths[b] outside [1, Lk] (reported by dma_check; clamped) */
+} dma_status_t;
+
+/*
+ * Workspace bytes needed by one call.  Prefill geometry: Lq == Lk == L.
+ * Decode geometry: Lq == 1, Lk = cache length.  Returns 0 for any other
+ * geometry or unsupported sizes.
+ */
+DMA_API size_t dma_workspace_size(int B, int Lq, int Lk, int Hq, int Hkv, int d, int keep_window_size);
+
+/*
+ * S1, [DMA step 3]: dt = exp(A * softplus(dt_proj(value_states))), in float32.
+ *   v       [B, L, Hkv, d] bf16 value states
+ *   W_dt    [Hkv*d, Hkv] float32, A [Hkv] float32
+ *   dt_out  [B, Hkv, L] float32 (written)
+ */
+DMA_API dma_status_t dma_dt_scores(const void* v, const float* W_dt, const float* A, int B, int L, int Hkv, int d,
+                           float* dt_out, dma_stream_t stream);
+
+/*
+ * S2, [DMA step 3] prepare_dynamic_mask: for every (b, g, query row) the kept
+ * key set.  A row sees the keys a causal mask and the padding leave it (query
+ * row i of a prefill sees keys j <= i, j < len_b; the decode query sits at
+ * position len_b - 1 and sees keys j < len_b).  When Lk > keep_window_size the
+ * row keeps its keep_window_size best keys by dt (ties: lower key index);
+ * otherwise it keeps every key it sees.
+ *   dt           [B, Hkv, Lk] float32
+ *   Lq           Lk (prefill geometry) or 1 (decode geometry)
+ *   tau_out      [B, Hkv, Lq] uint64 or NULL.  tau = (bits(dt[j*]) << 32) | (0xFFFFFFFF - j*)
+ *                for the row's worst kept key j* when the top-k is active and the row
+ *                sees more than keep_window_size keys, else 0.  A seen key j is kept
+ *                iff (bits(dt[j]) << 32 | (0xFFFFFFFF - j)) >= tau.
+ *   bitmask_out  [B, Hkv, Lq, ceil(Lk/32)] uint32 or NULL: bit (j % 32) of word j / 32
+ *                is 1 iff key j is kept.  Expanded from the compact plan the
+ *                attention kernels read (debug/test use; it is Lq*Lk bits).
+ *   workspace    dma_workspace_size(B, Lq, Lk, Hkv, Hkv, 64, keep_window_size) bytes
+ *                or more; on return it holds the compact plan.
+ */
+DMA_API dma_status_t dma_build_mask(const float* dt, const int32_t* lengths, int B, int Hkv, int Lq, int Lk,
+                            int keep_window_size, uint64_t* tau_out, uint32_t* bitmask_out, void* workspace,
+                            size_t ws_bytes, dma_stream_t stream);
+
+/*
+ * S1 + S2 + S3, [DMA steps 3-4]: prefill attention with the dynamic mask.
+ * For query head h of kv group g and row i:
+ *   out[b, i, h, :] = sum_j p_j v[b, j, g, :],
+ *   p = softmax_fp32(scale * q[b, i, h, :] . k[b, j, g, :] + dt[b, g, j]) over the kept keys j.
+ *   dt_in   [B, Hkv, L] float32 or NULL; when given, S1 is skipped and dt_in is used.
+ *   scale   normally d^-0.5 ([DMA step 4]).
+ *   out     [B, L, Hq, d] bf16 (written; rows i >= len_b are computed with the same rule).
+ */
+DMA_API dma_status_t dma_forward_prefill(const void* q, const void* k, const void* v, const float* W_dt, const float* A,
+                                 const int32_t* lengths, int B, int L, int Hq, int Hkv, int d, int keep_window_size,
+                                 float scale, const float* dt_in, void* out, void* workspace, size_t ws_bytes,
+                                 dma_stream_t stream);
+
+/*
+ * S4, [DMA step 3 closing paragraph, step 4]: one decode step.  dt is computed
+ * over the whole cached value states, the query at position len_b - 1 keeps
+ * its keep_window_size best cached keys, and attends to them as above.
+ *   q       [B, Hq, d] bf16;  k_cache, v_cache [B, Lk, Hkv, d] bf16 (hold the current token)
+ *   dt_in   [B, Hkv, Lk] float32 or NULL
+ *   out     [B, Hq, d] bf16
+ */
+DMA_API dma_status_t dma_decode_step(const void* q, const void* k_cache, const void* v_cache, const float* W_dt,
+                             const float* A, const int32_t* lengths, int B, int Lk, int Hq, int Hkv, int d,
+                             int keep_window_size, float scale, const float* dt_in, void* out, void* workspace,
+                             size_t ws_bytes, dma_stream_t stream);
+
+/*
+ * Synchronises `stream`, then returns the status recorded in the workspace by
+ * the device (DMA_OK if none).  clear != 0 resets the word afterwards.
+ */
+DMA_API dma_status_t dma_check(void* workspace, int clear, dma_stream_t stream);
+
+/*
+ * Profiling aid.  events: caller-owned cudaEvent_t handles (created with
+ * timing enabled), n >= 4, or NULL to stop.  While set, on the calling host
+ * thread, dma_forward_prefill and dma_decode_step record events[0] before
+ * their first kernel, events[1] after S1 (dt), events[2] after S2 (selection)
+ * and events[3] after the attention, all on the call's stream.  The library
+ * keeps only the pointer; the caller keeps the array alive while it is set.
+ */
+DMA_API dma_status_t dma_set_stage_events(void* const* events, int n);
+
+/* Human-readable name of a status. Never NULL. */
+DMA_API const char* dma_status_string(dma_status_t status);
+
+/* The cudaError_t of the last DMA_ERR_CUDA returned on this thread (0 if none). */
+DMA_API int dma_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DMA_H_ */

@@ -73,6 +73,24 @@ def decode_bytes(wl, lengths):
 
 
 # ----------------------------------------------------------------------------
+# multi-rank aggregation (weak scaling: every rank runs its own copy)
+# ----------------------------------------------------------------------------
+
+def max_over_ranks(v, dist=None, device=None):
+    """Largest value over all ranks (timings are reported as the slowest rank)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(v)
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(units_per_rank, ms_max, world):
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return world * units_per_rank / (ms_max * 1e-3)
+
+
+# ----------------------------------------------------------------------------
 # helpers
 # ----------------------------------------------------------------------------
 
@@ -295,12 +313,8 @@ def run_ours(args):
             pg.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(v):
-        if pg is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
+    def rank_max(v):
+        return max_over_ranks(v, pg, dev)
 
     peaks = load_peaks()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -309,9 +323,9 @@ def run_ours(args):
     with ClockSampler(local) as clk:
         head = time_prefill(dma, wl, args.steps, args.warmup, flush, dev, ranks_sync)
     clocks = clk.summary()
-    ms = max_over_ranks(head["ms"])
-    att_ms = max_over_ranks(head["stage_ms"][2])
-    value = world * head["flops"] / (ms * 1e-3) / 1e12
+    ms = rank_max(head["ms"])
+    att_ms = rank_max(head["stage_ms"][2])
+    value = aggregate_throughput(head["flops"], ms, world) / 1e12
     att_tflops = head["flops"] / (att_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "kernel": "attn_prefill_kernel<64>", "achieved": round(att_tflops, 2),
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
@@ -336,9 +350,9 @@ def run_ours(args):
     if not args.quick:
         for name in ("sparse_pad", "long"):
             o = time_prefill(dma, WORKLOADS[name], args.steps, args.warmup, flush, dev, ranks_sync)
-            oms = max_over_ranks(o["ms"])
-            a_ms = max_over_ranks(o["stage_ms"][2])
-            others[name] = {"value": round(o["flops"] / (oms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            oms = rank_max(o["ms"])
+            a_ms = rank_max(o["stage_ms"][2])
+            others[name] = {"value": round(aggregate_throughput(o["flops"], oms, world) / 1e12, 3), "unit": "TFLOP/s",
                             "ms_per_step": round(oms, 5),
                             "attention_tflops": round(o["flops"] / (a_ms * 1e-3) / 1e12, 2),
                             "attention_frac": round(o["flops"] / (a_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
@@ -347,8 +361,8 @@ def run_ours(args):
             del o
             torch.cuda.empty_cache()
         d = time_decode(dma, WORKLOADS["decode"], args.steps, args.warmup, flush, dev, ranks_sync)
-        dms = max_over_ranks(d["ms"])
-        dt_ms = max_over_ranks(d["stage_ms"][0])
+        dms = rank_max(d["ms"])
+        dt_ms = rank_max(d["stage_ms"][0])
         gbs = d["bytes"] / (dms * 1e-3) / 1e9
         v_scan = WORKLOADS["decode"].B * WORKLOADS["decode"].L * WORKLOADS["decode"].Hkv * WORKLOADS["decode"].d * 2
         others["decode"] = {"value": round(world * gbs, 1), "unit": "GB/s", "ms_per_step": round(dms, 5),

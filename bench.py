@@ -294,6 +294,25 @@ def cpu_baseline_prefill(wl, x, budget_s=12.0):
                       f"(dt of the whole sequence included), {dt_s:.1f} s"}
 
 
+def run_only(args):
+    """One workload, timed with the same rules, for profiler command lines."""
+    from doge_dynamic_mask_b200 import dma
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    wl = WORKLOADS[args.only]
+    if args.batch:
+        wl = wl.replace(B=args.batch)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    if wl.mode == "prefill":
+        r = time_prefill(dma, wl, args.steps, args.warmup, flush, dev, torch.cuda.synchronize)
+        line = {"workload": wl.name, "B": wl.B, "value": r["flops"] / (r["ms"] * 1e-3) / 1e12, "unit": "TFLOP/s"}
+    else:
+        r = time_decode(dma, wl, args.steps, args.warmup, flush, dev, torch.cuda.synchronize)
+        line = {"workload": wl.name, "B": wl.B, "value": r["bytes"] / (r["ms"] * 1e-3) / 1e9, "unit": "GB/s"}
+    line.update({"ms_per_step": r["ms"], "stage_ms": r["stage_ms"], "gpu_launches": r["launches"]})
+    print(json.dumps(line), flush=True)
+
+
 def run_ours(args):
     from doge_dynamic_mask_b200 import dma
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -420,11 +439,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="headline workload only")
+    ap.add_argument("--only", choices=sorted(WORKLOADS), help="time one workload only (profiling)")
+    ap.add_argument("--batch", type=int, default=0, help="with --only: override the batch size")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.only:
+        run_only(args)
     else:
         run_ours(args)
 

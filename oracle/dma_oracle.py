@@ -147,6 +147,16 @@ def composite_key(dt_value, j):
     return (bits << 32) | (0xFFFFFFFF - int(j))
 
 
+def threshold_row(dt_row, len_b, Lq, Lk, w, i):
+    """tau of one query row (see thresholds)."""
+    lim = _valid_limit(i, len_b, Lq, Lk)
+    if Lk > w and lim > w:
+        order = np.argsort(-np.asarray(dt_row[:lim], dtype=np.float64), kind="stable")
+        j = int(order[w - 1])
+        return composite_key(dt_row[j], j)
+    return 0
+
+
 def thresholds(dt, lengths, Lq, Lk, w):
     """Row thresholds tau [B, H_kv, Lq] as uint64.
 
@@ -160,11 +170,7 @@ def thresholds(dt, lengths, Lq, Lk, w):
     for b in range(B):
         for g in range(Hkv):
             for i in range(Lq):
-                lim = _valid_limit(i, int(lengths[b]), Lq, Lk)
-                if Lk > w and lim > w:
-                    order = np.argsort(-dt[b, g, :lim].astype(np.float64), kind="stable")
-                    j = int(order[w - 1])
-                    tau[b, g, i] = composite_key(dt[b, g, j], j)
+                tau[b, g, i] = threshold_row(dt[b, g], int(lengths[b]), Lq, Lk, w, i)
     return tau
 
 

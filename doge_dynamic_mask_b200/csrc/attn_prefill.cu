@@ -282,26 +282,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         DMA_TMEM_LD32(tS + 64, (r + 64));
         DMA_TMEM_LD32(tS + 96, (r + 96));
         tmem_wait_ld();
-        const float* mb = reinterpret_cast<const float*>(sMeta + s * C::kMetaBytes);
-        const uint32_t* ms = reinterpret_cast<const uint32_t*>(sMeta + s * C::kMetaBytes + kKeyTile * 4);
+        // dt bias (log2 units) and row intervals of this key tile.  The table is
+        // read 16 columns at a time, each group's address chained through the
+        // previous group's result so the loads are not all hoisted (register
+        // pressure: the whole S row is live here).
+        const float4* mb4 = reinterpret_cast<const float4*>(sMeta + s * C::kMetaBytes);
+        const uint4* ms4 = reinterpret_cast<const uint4*>(sMeta + s * C::kMetaBytes + kKeyTile * 4);
         const bool full = (j + 1) * kKeyTile <= n_full || !row_valid;
         float tmax = -INFINITY;
         if (full) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const float x = fmaf(__uint_as_float(r[c]), scale_log2, mb[c]);
-            r[c] = __float_as_uint(x);
-            tmax = fmaxf(tmax, x);
+          for (int g16 = 0; g16 < 8; ++g16) {
+            const float4* gp = mb4 + g16 * 4;
+            asm volatile("" : "+l"(gp) : "f"(tmax));
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const float4 bb = gp[q4];
+              const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int c = g16 * 16 + q4 * 4 + e;
+                const float x = fmaf(__uint_as_float(r[c]), scale_log2, bv[e]);
+                r[c] = __float_as_uint(x);
+                tmax = fmaxf(tmax, x);
+              }
+            }
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const uint32_t sp = ms[c];
-            const bool kept = static_cast<uint32_t>(row - static_cast<int>(sp & 0xFFFFu)) <
-                              ((sp >> 16) - (sp & 0xFFFFu));
-            const float x = kept ? fmaf(__uint_as_float(r[c]), scale_log2, mb[c]) : -INFINITY;
-            r[c] = __float_as_uint(x);
-            tmax = fmaxf(tmax, x);
+          for (int g16 = 0; g16 < 8; ++g16) {
+            const float4* gp = mb4 + g16 * 4;
+            const uint4* gs = ms4 + g16 * 4;
+            asm volatile("" : "+l"(gp), "+l"(gs) : "f"(tmax));
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const float4 bb = gp[q4];
+              const uint4 ss = gs[q4];
+              const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+              const uint32_t sv[4] = {ss.x, ss.y, ss.z, ss.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int c = g16 * 16 + q4 * 4 + e;
+                const uint32_t sp = sv[e];
+                const bool kept = static_cast<uint32_t>(row - static_cast<int>(sp & 0xFFFFu)) <
+                                  ((sp >> 16) - (sp & 0xFFFFu));
+                const float x = kept ? fmaf(__uint_as_float(r[c]), scale_log2, bv[e]) : -INFINITY;
+                r[c] = __float_as_uint(x);
+                tmax = fmaxf(tmax, x);
+              }
+            }
           }
         }
         const float m_new = fmaxf(m, tmax);
@@ -313,17 +342,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float m_use = m == -INFINITY ? 0.0f : m;
         float rs = 0.0f;
-        uint32_t pk[64];
+        // P in two halves of 64 keys (32 packed columns each): fewer live registers
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float p0 = fast_exp2(__uint_as_float(r[2 * c]) - m_use);
-          const float p1 = fast_exp2(__uint_as_float(r[2 * c + 1]) - m_use);
-          rs += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float p0 = fast_exp2(__uint_as_float(r[64 * half + 2 * c]) - m_use);
+            const float p1 = fast_exp2(__uint_as_float(r[64 * half + 2 * c + 1]) - m_use);
+            rs += p0 + p1;
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+          DMA_TMEM_ST32(tS + 32 * half, pk);
         }
         l += rs;
-        DMA_TMEM_ST32(tS + 0, (pk + 0));
-        DMA_TMEM_ST32(tS + 32, (pk + 32));
         if (j > 0) {
           // consume every o_done phase in order (PV of the previous tile), so
           // the parity of the epilogue's wait is never ambiguous

@@ -6,27 +6,24 @@
 // scalar per kv head).  No bias: attention_bias=False in section
 // "DogeConfig 全参数详解".
 //
-// Design.  The projection is a skinny GEMV: every token row of Hkv*d bf16
-// values meets the same [Hkv*d, Hkv] weight, so the kernel is bound by the one
-// read of V from HBM.  Each thread owns one 16-byte chunk (8 channels) of the
-// token row for the whole kernel and keeps those 8 x Hkv weights in
-// registers; it streams many tokens, accumulating Hkv partial sums per token
-// with packed f32x2 FMAs.  The R = Hkv*d/8 threads sharing a token combine
-// their partials with a butterfly reduce-scatter inside the warp (Hkv values
-// shrink to one per lane in log2(Hkv) shuffle stages) and, when a row spans
-// several warps, a tiny shared-memory sum.  The epilogue applies softplus, the
-// A multiply and exp in float32 and writes dt [B, Hkv, L] coalesced.
+// Design.  The projection is a skinny GEMV: every token row of C = Hkv*d bf16
+// values meets the same [C, Hkv] weight, so the kernel is bound by the one read
+// of V from HBM.  Each lane owns whole tokens (K of them): it streams its rows
+// in 16-byte chunks (8 channels), keeps DEPTH chunks per token in flight in
+// registers, and accumulates all Hkv dot products itself, so there is no
+// cross-lane reduction and no block barrier in the main loop.  The weight is
+// staged once per block in shared memory as channel pairs
+// (W[2p][g], W[2p+1][g]); all lanes of a warp read the same chunk's weights at
+// the same time (broadcast), and each pair feeds one packed fma.rn.f32x2 with
+// the matching pair of value channels.  The epilogue adds the two halves,
+// applies softplus, the A multiply and exp in float32 and writes dt
+// [B, Hkv, L] coalesced across lanes.
 #include "common.cuh"
 
 namespace dma {
 namespace {
 
 constexpr int kDtThreads = 256;
-
-__device__ __forceinline__ void bf16x2_to_f32(uint32_t u, float& lo, float& hi) {
-  lo = __uint_as_float(u << 16);
-  hi = __uint_as_float(u & 0xFFFF0000u);
-}
 
 __device__ __forceinline__ unsigned long long pack_f32x2(float lo, float hi) {
   unsigned long long r;
@@ -40,137 +37,130 @@ __device__ __forceinline__ void unpack_f32x2(unsigned long long v, float& lo, fl
 __device__ __forceinline__ void fma_f32x2(unsigned long long& acc, unsigned long long a, unsigned long long b) {
   asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
 }
+// Two bf16 (low half first) as a float32 pair.
+__device__ __forceinline__ unsigned long long bf16x2_to_f32x2(uint32_t u) {
+  return pack_f32x2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
 
 __device__ __forceinline__ float softplus_f32(float x) {
   // log(1 + e^x) in the overflow-free form max(x, 0) + log1p(e^-|x|).
   return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
 }
 
-// HKV outputs per token; R = HKV*D/8 threads share one token row.
-template <int HKV, int D, int UNROLL>
+__device__ __forceinline__ uint32_t word(const uint4& u, int i) {
+  return i == 0 ? u.x : i == 1 ? u.y : i == 2 ? u.z : u.w;
+}
+
+// HKV outputs per token, D head dims, K tokens per lane, DEPTH chunks in flight.
+template <int HKV, int D, int K, int DEPTH>
 __global__ void __launch_bounds__(kDtThreads) dt_scores_kernel(const uint4* __restrict__ v,
                                                                 const float* __restrict__ W,
                                                                 const float* __restrict__ A, long long ntok,
                                                                 int L, float* __restrict__ dt) {
-  constexpr int R = HKV * D / 8;                   // chunks (threads) per token row
-  constexpr int TS = kDtThreads / R;               // tokens per step (>= 1)
-  constexpr int TB = TS * UNROLL;                  // tokens per block iteration
-  constexpr int RW = R < 32 ? R : 32;              // lanes of one warp sharing a token
-  constexpr int NPART = R > 32 ? R / 32 : 1;       // warps sharing a token
-  static_assert(kDtThreads % R == 0, "row must tile the block");
+  constexpr int C = HKV * D;          // channels per token
+  constexpr int NCH = C / 8;          // 16-byte chunks per token
+  static_assert(NCH % DEPTH == 0, "chunk ring must tile the row");
+  extern __shared__ unsigned long long w2s[];   // [C/2][HKV] channel pairs
 
-  __shared__ float part[NPART][TB][HKV];
-
-  const int tid = threadIdx.x;
-  const int c = tid % R;                            // chunk of the row owned by this thread
-  const int slot = tid / R;                         // token slot within a step
-  const int lane = tid & 31;
-
-  // weights of this thread's 8 channels, packed in f32x2 pairs over outputs
-  constexpr int HP = HKV >= 2 ? HKV / 2 : 1;
-  unsigned long long w2[8][HP];
-#pragma unroll
-  for (int e = 0; e < 8; ++e)
-#pragma unroll
-    for (int i = 0; i < HP; ++i)
-      w2[e][i] = HKV >= 2 ? pack_f32x2(W[(c * 8 + e) * HKV + 2 * i], W[(c * 8 + e) * HKV + 2 * i + 1])
-                          : pack_f32x2(W[c * 8 + e], 0.0f);
-
-  const long long n_iter = (ntok + TB - 1) / TB;
-  for (long long it = blockIdx.x; it < n_iter; it += gridDim.x) {
-    const long long tok0 = it * TB;
-    uint4 buf[UNROLL];
-#pragma unroll
-    for (int s = 0; s < UNROLL; ++s) {
-      const long long t = tok0 + slot + s * TS;
-      buf[s] = t < ntok ? v[t * R + c] : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int s = 0; s < UNROLL; ++s) {
-      float x[8];
-      bf16x2_to_f32(buf[s].x, x[0], x[1]);
-      bf16x2_to_f32(buf[s].y, x[2], x[3]);
-      bf16x2_to_f32(buf[s].z, x[4], x[5]);
-      bf16x2_to_f32(buf[s].w, x[6], x[7]);
-      unsigned long long acc2[HP];
-#pragma unroll
-      for (int i = 0; i < HP; ++i) acc2[i] = 0ull;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const unsigned long long xx = pack_f32x2(x[e], x[e]);
-#pragma unroll
-        for (int i = 0; i < HP; ++i) fma_f32x2(acc2[i], xx, w2[e][i]);
-      }
-      float acc[HKV];
-#pragma unroll
-      for (int i = 0; i < HP; ++i) {
-        float lo, hi;
-        unpack_f32x2(acc2[i], lo, hi);
-        acc[2 * i < HKV ? 2 * i : 0] = lo;
-        if (2 * i + 1 < HKV) acc[2 * i + 1] = hi;
-      }
-
-      // butterfly reduce-scatter over the RW lanes sharing this token: each
-      // split stage halves the outputs a lane holds (kLogH stages), then plain
-      // xor stages sum over the remaining lanes.
-      constexpr int kLogH = HKV >= 16 ? 4 : HKV >= 8 ? 3 : HKV >= 4 ? 2 : HKV >= 2 ? 1 : 0;
-      static_assert((1 << kLogH) == HKV && HKV <= RW, "outputs must fit the lanes of a row");
-      int gbase = 0;
-#pragma unroll
-      for (int st = 0; st < kLogH; ++st) {
-        const int o = RW >> (st + 1);
-        const int half = HKV >> (st + 1);
-        const bool upper = (lane & o) != 0;
-#pragma unroll
-        for (int i = 0; i < half; ++i) {
-          const float send = upper ? acc[i] : acc[i + half];
-          const float keep = upper ? acc[i + half] : acc[i];
-          acc[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
-        }
-        if (upper) gbase += half;
-      }
-#pragma unroll
-      for (int o = RW >> (kLogH + 1); o >= 1; o >>= 1) acc[0] += __shfl_xor_sync(0xFFFFFFFFu, acc[0], o);
-      // one lane per output (low plain-stage lane bits clear) writes the warp's partial
-      constexpr int kPlainMask = (RW >> kLogH) - 1;
-      if ((lane & kPlainMask) == 0) {
-        const int p = NPART > 1 ? (tid / 32) % NPART : 0;
-        part[p][slot + s * TS][gbase] = acc[0];
-      }
-    }
-    __syncthreads();
-    for (int i = tid; i < TB * HKV; i += kDtThreads) {
-      const int g = i / TB;
-      const int tl = i % TB;
-      const long long t = tok0 + tl;
-      if (t < ntok) {
-        float x = 0.0f;
-#pragma unroll
-        for (int p = 0; p < NPART; ++p) x += part[p][tl][g];
-        const float y = expf(A[g] * softplus_f32(x));
-        const long long b = t / L;
-        const long long l = t - b * L;
-        dt[(b * HKV + g) * L + l] = y;
-      }
-    }
-    __syncthreads();
+  for (int i = threadIdx.x; i < (C / 2) * HKV; i += kDtThreads) {
+    const int p = i / HKV, g = i % HKV;
+    w2s[i] = pack_f32x2(W[(2 * p) * HKV + g], W[(2 * p + 1) * HKV + g]);
   }
+  __syncthreads();
+
+  const int lane = threadIdx.x & 31;
+  const long long warp_global = static_cast<long long>(blockIdx.x) * (kDtThreads / 32) + (threadIdx.x >> 5);
+  const long long nwarps = static_cast<long long>(gridDim.x) * (kDtThreads / 32);
+  const long long per_warp = 32LL * K;
+  for (long long base = warp_global * per_warp; base < ntok; base += nwarps * per_warp) {
+    long long tok[K];
+    bool live[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      tok[k] = base + k * 32 + lane;
+      live[k] = tok[k] < ntok;
+    }
+    unsigned long long acc[K][HKV];
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+#pragma unroll
+      for (int g = 0; g < HKV; ++g) acc[k][g] = 0ull;
+
+    uint4 ring[DEPTH][K];
+#pragma unroll
+    for (int s = 0; s < DEPTH; ++s)
+#pragma unroll
+      for (int k = 0; k < K; ++k)
+        ring[s][k] = live[k] ? __ldcs(v + tok[k] * NCH + s) : make_uint4(0, 0, 0, 0);
+
+#pragma unroll 1
+    for (int ch0 = 0; ch0 < NCH; ch0 += DEPTH) {
+#pragma unroll
+      for (int s = 0; s < DEPTH; ++s) {
+        const int ch = ch0 + s;
+        uint4 cur[K];
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+          cur[k] = ring[s][k];
+          const int nx = ch + DEPTH;
+          ring[s][k] = (live[k] && nx < NCH) ? __ldcs(v + tok[k] * NCH + nx) : make_uint4(0, 0, 0, 0);
+        }
+        const unsigned long long* wc = w2s + static_cast<size_t>(ch) * 4 * HKV;   // this chunk's 4 pairs
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) {
+          unsigned long long wp[HKV];
+#pragma unroll
+          for (int g = 0; g < HKV; ++g) wp[g] = wc[pp * HKV + g];
+#pragma unroll
+          for (int k = 0; k < K; ++k) {
+            const unsigned long long xp = bf16x2_to_f32x2(word(cur[k], pp));
+#pragma unroll
+            for (int g = 0; g < HKV; ++g) fma_f32x2(acc[k][g], xp, wp[g]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      if (!live[k]) continue;
+      const long long b = tok[k] / L;
+      const long long l = tok[k] - b * L;
+#pragma unroll
+      for (int g = 0; g < HKV; ++g) {
+        float lo, hi;
+        unpack_f32x2(acc[k][g], lo, hi);
+        dt[(b * HKV + g) * L + l] = expf(A[g] * softplus_f32(lo + hi));
+      }
+    }
+  }
+}
+
+template <int HKV, int D, int K>
+cudaError_t launch_k(const void* v, const float* W, const float* A, long long ntok, int L, float* dt, int nsm,
+                     cudaStream_t s) {
+  constexpr int DEPTH = 4;
+  const size_t smem = static_cast<size_t>(HKV) * D / 2 * HKV * sizeof(unsigned long long);
+  auto kern = dt_scores_kernel<HKV, D, K, DEPTH>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const long long warps_needed = (ntok + 32LL * K - 1) / (32LL * K);
+  long long blocks = (warps_needed + kDtThreads / 32 - 1) / (kDtThreads / 32);
+  const long long cap = 4LL * nsm;
+  if (blocks > cap) blocks = cap;
+  kern<<<static_cast<int>(blocks), kDtThreads, smem, s>>>(static_cast<const uint4*>(v), W, A, ntok, L, dt);
+  return cudaGetLastError();
 }
 
 template <int HKV, int D>
 cudaError_t launch_t(const void* v, const float* W, const float* A, int B, int L, float* dt, cudaStream_t s) {
-  constexpr int R = HKV * D / 8;
-  constexpr int UNROLL = 8;
-  constexpr int TB = (kDtThreads / R) * UNROLL;
+  constexpr int KBIG = HKV >= 8 ? 2 : 4;
   const long long ntok = static_cast<long long>(B) * L;
-  const long long n_iter = (ntok + TB - 1) / TB;
   int dev = 0, nsm = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  const long long grid = n_iter < 4LL * nsm ? n_iter : 4LL * nsm;
-  dt_scores_kernel<HKV, D, UNROLL><<<static_cast<int>(grid), kDtThreads, 0, s>>>(
-      static_cast<const uint4*>(v), W, A, ntok, L, dt);
-  return cudaGetLastError();
+  // short inputs: one token per lane so that every SM gets warps
+  if (ntok < 32LL * KBIG * 8 * 2 * nsm) return launch_k<HKV, D, 1>(v, W, A, ntok, L, dt, nsm, s);
+  return launch_k<HKV, D, KBIG>(v, W, A, ntok, L, dt, nsm, s);
 }
 
 }  // namespace

@@ -55,7 +55,7 @@ def test_prefill_full_size_sampled(dma, name, heads):
         rows = sample_rows(wl.L, int(lengths[b]), wl.w, rng)
         # tau of the sampled rows, bit-exact, from the same float32 dt
         tau = torch.empty((1, wl.Hkv, wl.L), dtype=torch.int64, device="cuda")
-        dma.dma_build_mask(torch.from_numpy(dt).cuda(), x["lengths"][b:b + 1], wl.L, wl.w, tau_out=tau)
+        dma.dma_build_mask(torch.from_numpy(dt).cuda(), x["lengths"][b:b + 1].clone(), wl.L, wl.w, tau_out=tau)
         got_tau = tau.cpu().numpy().view(np.uint64)
         for g in sorted({h // (wl.Hq // wl.Hkv) for h in heads}):
             for i in rows:

@@ -10,9 +10,11 @@
 // w + 127 keys any of its rows keeps; the kernel streams those keys in tiles of
 // 128 and never touches a key the tile does not keep.
 //   * warp 0 (producer): TMA loads the two Q tiles once, then for every key
-//     tile gathers the 128 listed K rows and V rows with tile::gather4 (four
-//     rows per instruction, 128-byte swizzle) into a ring of shared-memory
-//     stages, and copies the tile's dt bias and row intervals next to them.
+//     tile fetches the 128 listed K rows and V rows into a ring of
+//     shared-memory stages (128-byte swizzle): one box copy per 64-column slab
+//     when the listed keys are one ascending run, else tile::gather4 (four
+//     listed rows per instruction); it copies the tile's dt bias and row
+//     intervals next to them.
 //   * warp 1 (one thread): issues tcgen05.mma.  S_h = Q_h K^T (M=128, N=128,
 //     K=d) into TMEM, and O_h += P_h V (A = P read from TMEM, B = V from shared
 //     memory, N=d).  The two heads ping-pong: while one head's softmax runs the
@@ -72,7 +74,8 @@ __device__ __forceinline__ bool aborted(volatile int* flag) { return *flag != 0;
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-                        const __grid_constant__ CUtensorMap tmap_v, PrefillPlan plan, int B, int L, int Hq,
+                        const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_k3,
+                        const __grid_constant__ CUtensorMap tmap_v3, PrefillPlan plan, int B, int L, int Hq,
                         int Hkv, float scale_log2, uint16_t* __restrict__ out, uint32_t* err) {
   using C = Cfg<D>;
   extern __shared__ unsigned char smem_raw[];
@@ -126,6 +129,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmap_q);
     prefetch_tmap(&tmap_k);
     prefetch_tmap(&tmap_v);
+    prefetch_tmap(&tmap_k3);
+    prefetch_tmap(&tmap_v3);
   }
   if (warp == 2) tmem_alloc(tmem_slot, C::kTmemCols);
   tc_fence_before();
@@ -149,6 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   b * L + r0);
     }
     const int32_t* idx_t = plan.idx + tile * plan.cap;
+    const int32_t* kbase_t = plan.kbase + tile * (plan.cap / kKeyTile);
     const float* bias_t = plan.bias + tile * plan.cap;
     const uint32_t* span_t = plan.span + tile * plan.cap;
     for (int j = 0; j < n_kt; ++j) {
@@ -162,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (aborted(abort_flag)) break;
       const int e = j * kKeyTile + lane * 4;
-      const int4 ix = *reinterpret_cast<const int4*>(idx_t + e);
+      const int kb0 = kbase_t[j];
       const float4 bi = *reinterpret_cast<const float4*>(bias_t + e);
       const uint4 sp = *reinterpret_cast<const uint4*>(span_t + e);
       float* mb = reinterpret_cast<float*>(sMeta + s * C::kMetaBytes);
@@ -171,23 +177,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           make_float4(bi.x * kLog2e, bi.y * kLog2e, bi.z * kLog2e, bi.w * kLog2e);
       *reinterpret_cast<uint4*>(ms + lane * 4) = sp;
       const int base_row = b * L;
-      const int r_0 = (base_row + ix.x) * Hkv + g;
-      const int r_1 = (base_row + ix.y) * Hkv + g;
-      const int r_2 = (base_row + ix.z) * Hkv + g;
-      const int r_3 = (base_row + ix.w) * Hkv + g;
       __syncwarp();
-      if (lane == 0) mbar_arrive_expect_tx(bars.k_full + s, C::kKVBytes);
-      __syncwarp();
+      if (kb0 >= 0) {
+        // one ascending run of keys: a 128-row box per 64-column slab
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bars.k_full + s, C::kKVBytes);
 #pragma unroll
-      for (int sl = 0; sl < C::kSlabs; ++sl)
-        tma_gather4(sK + s * C::kKVBytes + sl * C::kSlabBytes + lane * 512, &tmap_k, bars.k_full + s, sl * 64,
-                    r_0, r_1, r_2, r_3);
-      if (lane == 0) mbar_arrive_expect_tx(bars.v_full + s, C::kKVBytes);
-      __syncwarp();
+          for (int sl = 0; sl < C::kSlabs; ++sl)
+            tma_load_3d(sK + s * C::kKVBytes + sl * C::kSlabBytes, &tmap_k3, bars.k_full + s, sl * 64, g,
+                        base_row + kb0);
+          mbar_arrive_expect_tx(bars.v_full + s, C::kKVBytes);
 #pragma unroll
-      for (int sl = 0; sl < C::kSlabs; ++sl)
-        tma_gather4(sV + s * C::kKVBytes + sl * C::kSlabBytes + lane * 512, &tmap_v, bars.v_full + s, sl * 64,
-                    r_0, r_1, r_2, r_3);
+          for (int sl = 0; sl < C::kSlabs; ++sl)
+            tma_load_3d(sV + s * C::kKVBytes + sl * C::kSlabBytes, &tmap_v3, bars.v_full + s, sl * 64, g,
+                        base_row + kb0);
+        }
+      } else {
+        const int4 ix = *reinterpret_cast<const int4*>(idx_t + e);
+        const int r_0 = (base_row + ix.x) * Hkv + g;
+        const int r_1 = (base_row + ix.y) * Hkv + g;
+        const int r_2 = (base_row + ix.z) * Hkv + g;
+        const int r_3 = (base_row + ix.w) * Hkv + g;
+        if (lane == 0) mbar_arrive_expect_tx(bars.k_full + s, C::kKVBytes);
+        __syncwarp();
+#pragma unroll
+        for (int sl = 0; sl < C::kSlabs; ++sl)
+          tma_gather4(sK + s * C::kKVBytes + sl * C::kSlabBytes + lane * 512, &tmap_k, bars.k_full + s, sl * 64,
+                      r_0, r_1, r_2, r_3);
+        if (lane == 0) mbar_arrive_expect_tx(bars.v_full + s, C::kKVBytes);
+        __syncwarp();
+#pragma unroll
+        for (int sl = 0; sl < C::kSlabs; ++sl)
+          tma_gather4(sV + s * C::kKVBytes + sl * C::kSlabBytes + lane * 512, &tmap_v, bars.v_full + s, sl * 64,
+                      r_0, r_1, r_2, r_3);
+      }
       issued = j + 1;
     }
     // drain: every copy issued must have landed before the CTA can leave
@@ -459,12 +482,24 @@ cudaError_t launch_d(const void* q, const void* k, const void* v, const Geometry
   }
   const void* kv[2] = {k, v};
   CUtensorMap* maps[2] = {&tk, &tv};
+  CUtensorMap tk3, tv3;
+  CUtensorMap* maps3[2] = {&tk3, &tv3};
   for (int i = 0; i < 2; ++i) {
+    // rows (b, j, g) of [B*L*Hkv, d], fetched four listed rows at a time
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), BL * g.Hkv};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
     cuuint32_t box[2] = {64, 1};
     cuuint32_t es[2] = {1, 1};
     if (enc(maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kv[i]), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    // [B*L, Hkv, d]: 128 consecutive keys of one kv head per box
+    cuuint64_t dims3[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(g.Hkv), BL};
+    cuuint64_t strides3[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(g.Hkv) * D * 2};
+    cuuint32_t box3[3] = {64, 1, static_cast<cuuint32_t>(kKeyTile)};
+    cuuint32_t es3[3] = {1, 1, 1};
+    if (enc(maps3[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kv[i]), dims3, strides3, box3, es3,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
@@ -476,7 +511,7 @@ cudaError_t launch_d(const void* q, const void* k, const void* v, const Geometry
   const int npairs = (nrep + 1) / 2;
   const long long nblocks = static_cast<long long>(plan.n_row_tiles) * g.B * g.Hkv * npairs;
   attn_prefill_kernel<D><<<static_cast<unsigned>(nblocks), kThreads, C::kSmemBytes, s>>>(
-      tq, tk, tv, plan, g.B, g.Lk, g.Hq, g.Hkv, scale * kLog2e, static_cast<uint16_t*>(out), err);
+      tq, tk, tv, tk3, tv3, plan, g.B, g.Lk, g.Hq, g.Hkv, scale * kLog2e, static_cast<uint16_t*>(out), err);
   return cudaGetLastError();
 }
 

@@ -84,6 +84,7 @@ size_t prefill_plan_bytes(const Geometry& g) {
   off = align_up(off + tiles * cap * 4, 256);       // bias
   off = align_up(off + tiles * cap * 4, 256);       // span
   off = align_up(off + tiles * 8, 256);             // counts
+  off = align_up(off + tiles * (cap / kKeyTile) * 4, 256);   // kbase
   return off;
 }
 
@@ -106,6 +107,8 @@ PrefillPlan carve_prefill_plan(void* ws, const Geometry& g) {
   p.span = reinterpret_cast<uint32_t*>(base + off);
   off = align_up(off + tiles * cap * 4, 256);
   p.counts = reinterpret_cast<int2*>(base + off);
+  off = align_up(off + tiles * 8, 256);
+  p.kbase = reinterpret_cast<int32_t*>(base + off);
   p.cap = cap;
   p.n_row_tiles = nrt;
   return p;

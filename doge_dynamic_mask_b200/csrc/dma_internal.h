@@ -40,6 +40,8 @@ __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a -
 //   counts[tiles]     int2    (n_full, n_total); entries [0, n_full) are kept by
 //                             every row of the tile; entries past n_total up to
 //                             the next multiple of kKeyTile are padding (span 0).
+//   kbase[tiles][cap / kKeyTile] int32  j0 when the key tile's listed keys are
+//                             exactly j0, j0+1, ... (in list order), else -1
 // tiles are ordered ((b * Hkv + g) * n_row_tiles + t).
 struct PrefillPlan {
   float* dt;        // [B, Hkv, L]
@@ -48,6 +50,7 @@ struct PrefillPlan {
   float* bias;
   uint32_t* span;
   int2* counts;
+  int32_t* kbase;
   int cap;          // entries per tile (multiple of kKeyTile)
   int n_row_tiles;
 };

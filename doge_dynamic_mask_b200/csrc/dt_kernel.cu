@@ -9,8 +9,8 @@
 // Design.  The projection is a skinny GEMV: every token row of C = Hkv*d bf16
 // values meets the same [C, Hkv] weight, so the kernel is bound by the one read
 // of V from HBM.  Each lane owns whole tokens (K of them): it streams its rows
-// in 16-byte chunks (8 channels), keeps DEPTH chunks per token in flight in
-// registers, and accumulates all Hkv dot products itself, so there is no
+// in 32-byte chunks (16 channels, one full sector per 256-bit load), keeps
+// DEPTH chunks per token in flight in registers, and accumulates all Hkv dot products itself, so there is no
 // cross-lane reduction and no block barrier in the main loop.  The weight is
 // staged once per block in shared memory as channel pairs
 // (W[2p][g], W[2p+1][g]); all lanes of a warp read the same chunk's weights at
@@ -51,14 +51,38 @@ __device__ __forceinline__ uint32_t word(const uint4& u, int i) {
   return i == 0 ? u.x : i == 1 ? u.y : i == 2 ? u.z : u.w;
 }
 
-// HKV outputs per token, D head dims, K tokens per lane, DEPTH chunks in flight.
-template <int HKV, int D, int K, int DEPTH>
+// 32 bytes (16 bf16 channels) of one token row.  WIDE: one 256-bit load (the
+// base pointer is 32-byte aligned); else two 128-bit loads.
+struct Chunk32 {
+  uint32_t w[8];
+};
+
+template <bool WIDE>
+__device__ __forceinline__ Chunk32 load_chunk(const uint4* __restrict__ v, long long idx16) {
+  Chunk32 c;
+  if constexpr (WIDE) {
+    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(c.w[0]), "=r"(c.w[1]), "=r"(c.w[2]), "=r"(c.w[3]), "=r"(c.w[4]), "=r"(c.w[5]),
+                   "=r"(c.w[6]), "=r"(c.w[7])
+                 : "l"(v + idx16));
+  } else {
+    const uint4 a = __ldcs(v + idx16), b = __ldcs(v + idx16 + 1);
+    c.w[0] = a.x; c.w[1] = a.y; c.w[2] = a.z; c.w[3] = a.w;
+    c.w[4] = b.x; c.w[5] = b.y; c.w[6] = b.z; c.w[7] = b.w;
+  }
+  return c;
+}
+
+// HKV outputs per token, D head dims, K tokens per lane, DEPTH 32-byte chunks
+// per token in flight.
+template <int HKV, int D, int K, int DEPTH, bool WIDE>
 __global__ void __launch_bounds__(kDtThreads) dt_scores_kernel(const uint4* __restrict__ v,
                                                                 const float* __restrict__ W,
                                                                 const float* __restrict__ A, long long ntok,
                                                                 int L, float* __restrict__ dt) {
   constexpr int C = HKV * D;          // channels per token
-  constexpr int NCH = C / 8;          // 16-byte chunks per token
+  constexpr int N16 = C / 8;          // 16-byte pieces per token
+  constexpr int NCH = C / 16;         // 32-byte chunks per token
   static_assert(NCH % DEPTH == 0, "chunk ring must tile the row");
   extern __shared__ unsigned long long w2s[];   // [C/2][HKV] channel pairs
 
@@ -86,34 +110,34 @@ __global__ void __launch_bounds__(kDtThreads) dt_scores_kernel(const uint4* __re
 #pragma unroll
       for (int g = 0; g < HKV; ++g) acc[k][g] = 0ull;
 
-    uint4 ring[DEPTH][K];
+    Chunk32 ring[DEPTH][K];
 #pragma unroll
     for (int s = 0; s < DEPTH; ++s)
 #pragma unroll
       for (int k = 0; k < K; ++k)
-        ring[s][k] = live[k] ? __ldcs(v + tok[k] * NCH + s) : make_uint4(0, 0, 0, 0);
+        if (live[k]) ring[s][k] = load_chunk<WIDE>(v, tok[k] * N16 + 2 * s);
 
 #pragma unroll 1
     for (int ch0 = 0; ch0 < NCH; ch0 += DEPTH) {
 #pragma unroll
       for (int s = 0; s < DEPTH; ++s) {
         const int ch = ch0 + s;
-        uint4 cur[K];
+        Chunk32 cur[K];
 #pragma unroll
         for (int k = 0; k < K; ++k) {
           cur[k] = ring[s][k];
           const int nx = ch + DEPTH;
-          ring[s][k] = (live[k] && nx < NCH) ? __ldcs(v + tok[k] * NCH + nx) : make_uint4(0, 0, 0, 0);
+          if (live[k] && nx < NCH) ring[s][k] = load_chunk<WIDE>(v, tok[k] * N16 + 2 * nx);
         }
-        const unsigned long long* wc = w2s + static_cast<size_t>(ch) * 4 * HKV;   // this chunk's 4 pairs
+        const unsigned long long* wc = w2s + static_cast<size_t>(ch) * 8 * HKV;   // this chunk's 8 pairs
 #pragma unroll
-        for (int pp = 0; pp < 4; ++pp) {
+        for (int pp = 0; pp < 8; ++pp) {
           unsigned long long wp[HKV];
 #pragma unroll
           for (int g = 0; g < HKV; ++g) wp[g] = wc[pp * HKV + g];
 #pragma unroll
           for (int k = 0; k < K; ++k) {
-            const unsigned long long xp = bf16x2_to_f32x2(word(cur[k], pp));
+            const unsigned long long xp = bf16x2_to_f32x2(cur[k].w[pp]);
 #pragma unroll
             for (int g = 0; g < HKV; ++g) fma_f32x2(acc[k][g], xp, wp[g]);
           }
@@ -135,12 +159,12 @@ __global__ void __launch_bounds__(kDtThreads) dt_scores_kernel(const uint4* __re
   }
 }
 
-template <int HKV, int D, int K>
+template <int HKV, int D, int K, bool WIDE>
 cudaError_t launch_k(const void* v, const float* W, const float* A, long long ntok, int L, float* dt, int nsm,
                      cudaStream_t s) {
-  constexpr int DEPTH = 4;
+  constexpr int DEPTH = 2;
   const size_t smem = static_cast<size_t>(HKV) * D / 2 * HKV * sizeof(unsigned long long);
-  auto kern = dt_scores_kernel<HKV, D, K, DEPTH>;
+  auto kern = dt_scores_kernel<HKV, D, K, DEPTH, WIDE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const long long warps_needed = (ntok + 32LL * K - 1) / (32LL * K);
@@ -158,9 +182,13 @@ cudaError_t launch_t(const void* v, const float* W, const float* A, int B, int L
   int dev = 0, nsm = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const bool wide = (reinterpret_cast<uintptr_t>(v) & 31u) == 0;
   // short inputs: one token per lane so that every SM gets warps
-  if (ntok < 32LL * KBIG * 8 * 2 * nsm) return launch_k<HKV, D, 1>(v, W, A, ntok, L, dt, nsm, s);
-  return launch_k<HKV, D, KBIG>(v, W, A, ntok, L, dt, nsm, s);
+  if (ntok < 32LL * KBIG * 8 * 2 * nsm)
+    return wide ? launch_k<HKV, D, 1, true>(v, W, A, ntok, L, dt, nsm, s)
+                : launch_k<HKV, D, 1, false>(v, W, A, ntok, L, dt, nsm, s);
+  return wide ? launch_k<HKV, D, KBIG, true>(v, W, A, ntok, L, dt, nsm, s)
+              : launch_k<HKV, D, KBIG, false>(v, W, A, ntok, L, dt, nsm, s);
 }
 
 }  // namespace

@@ -94,6 +94,8 @@ __global__ void __launch_bounds__(kSelThreads) select_prefill_kernel(const float
       bias_o[j] = 0.0f;
       span_o[j] = 0u;
     }
+    int32_t* kb = plan.kbase + tile * (plan.cap / kKeyTile);
+    for (int kt = tid; kt * kKeyTile < n_total; kt += blockDim.x) kb[kt] = kt * kKeyTile;   // [0, q] in order
     if (tid == 0) plan.counts[tile] = make_int2(n_full, n_total);
     return;
   }
@@ -206,6 +208,19 @@ __global__ void __launch_bounds__(kSelThreads) select_prefill_kernel(const float
     span_o[j] = 0u;
   }
   if (tid == 0) plan.counts[tile] = make_int2(n_full, n_total);
+  // key tiles whose listed keys are one ascending run j0, j0+1, ... can be
+  // fetched with a single box copy instead of a row gather
+  __syncthreads();
+  int32_t* kb = plan.kbase + tile * (plan.cap / kKeyTile);
+  const int lane = tid & 31;
+  for (int kt = tid >> 5; kt * kKeyTile < n_total; kt += blockDim.x >> 5) {
+    const int e0 = kt * kKeyTile;
+    const int j0 = idx_o[e0];
+    bool ok = true;
+    for (int e = e0 + lane; e < min(n_total, e0 + kKeyTile); e += 32) ok &= idx_o[e] == j0 + (e - e0);
+    ok = __all_sync(0xFFFFFFFFu, ok);
+    if (lane == 0) kb[kt] = ok ? j0 : -1;
+  }
 }
 
 __global__ void __launch_bounds__(kSelThreads) select_decode_kernel(const float* __restrict__ dt,

@@ -129,6 +129,36 @@ DMA_API dma_status_t dma_decode_step(const void* q, const void* k_cache, const v
                              size_t ws_bytes, dma_stream_t stream);
 
 /*
+ * dma_decode_step without a caller-provided workspace (the pages have no
+ * counterpart: this is a calling convention of this library).
+ *
+ * For callers that cannot allocate device memory themselves, for example code
+ * embedded in a framework that owns all device memory through its own pool
+ * and forbids raw cudaMalloc (which synchronises the device and fragments that
+ * pool), or plain C callers without a device allocator.  Inputs and outputs are
+ * still the caller's (same arguments and layouts as dma_decode_step); the
+ * scratch lives in a 64 MiB array inside this library's device memory, which
+ * every GPU that loads the library holds until the process exits.  This entry
+ * point calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - Returns DMA_ERR_WORKSPACE when the step needs more than 64 MiB of scratch,
+ *     i.e. when dma_workspace_size(B, 1, Lk, Hq, Hkv, d, keep_window_size)
+ *     exceeds 64 MiB (roughly B * Hkv * Lk above 15.7 million cached keys).
+ *   - The first call on a device looks up the array's device address on that
+ *     device (cudaGetSymbolAddress, with the device current); make that first
+ *     call before any stream capture.
+ *   - Every call on every stream shares the one array and it keeps the last
+ *     call's contents; calls that overlap on the GPU race, so serialise them
+ *     (one stream, or events).  The status word is cleared at the start of
+ *     each call; device-side faults are not reported back by this entry point
+ *     (lengths are still clamped), so use dma_decode_step with a workspace and
+ *     dma_check when you need that report.
+ */
+DMA_API dma_status_t dma_decode_step_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                             const float* W_dt, const float* A, const int32_t* lengths, int B, int Lk,
+                                             int Hq, int Hkv, int d, int keep_window_size, float scale,
+                                             const float* dt_in, void* out, dma_stream_t stream);
+
+/*
  * Synchronises `stream`, then returns the status recorded in the workspace by
  * the device (DMA_OK if none).  clear != 0 resets the word afterwards.
  */

@@ -235,7 +235,8 @@ dma_status_t dma_forward_prefill(const void* q, const void* k, const void* v, co
       (W_dt && !aligned16(W_dt)) || (A && !aligned16(A)) || (dt_in && !aligned16(dt_in)) ||
       (lengths && !aligned16(lengths)))
     return DMA_ERR_INVALID_ARG;
-  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return DMA_ERR_INVALID_ARG;
+  // the attention kernel carries the dt bias through the tensor core as dt / scale
+  if (!(scale >= 1.0e-20f && scale <= 1.0e20f)) return DMA_ERR_INVALID_ARG;
   dma_status_t st = check_shape(B, L, Hq, Hkv, d, keep_window_size);
   if (st != DMA_OK) return st;
   if ((st = device_ok()) != DMA_OK) return st;

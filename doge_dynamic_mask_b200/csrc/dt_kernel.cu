@@ -34,7 +34,7 @@ __device__ __forceinline__ void unpack_f32x2(unsigned long long v, float& lo, fl
   asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
 }
 // acc = a * b + acc on both float32 halves (round-to-nearest, like fmaf).
-__device__ __forceinline__ void fma_f32x2(unsigned long long& acc, unsigned long long a, unsigned long long b) {
+__device__ __forceinline__ void fma_acc_f32x2(unsigned long long& acc, unsigned long long a, unsigned long long b) {
   asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
 }
 // Two bf16 (low half first) as a float32 pair.
@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(kDtThreads) dt_scores_kernel(const uint4* __re
           for (int k = 0; k < K; ++k) {
             const unsigned long long xp = bf16x2_to_f32x2(cur[k].w[pp]);
 #pragma unroll
-            for (int g = 0; g < HKV; ++g) fma_f32x2(acc[k][g], xp, wp[g]);
+            for (int g = 0; g < HKV; ++g) fma_acc_f32x2(acc[k][g], xp, wp[g]);
           }
         }
       }

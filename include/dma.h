@@ -107,7 +107,8 @@ DMA_API dma_status_t dma_build_mask(const float* dt, const int32_t* lengths, int
  *   out[b, i, h, :] = sum_j p_j v[b, j, g, :],
  *   p = softmax_fp32(scale * q[b, i, h, :] . k[b, j, g, :] + dt[b, g, j]) over the kept keys j.
  *   dt_in   [B, Hkv, L] float32 or NULL; when given, S1 is skipped and dt_in is used.
- *   scale   normally d^-0.5 ([DMA step 4]).
+ *   scale   normally d^-0.5 ([DMA step 4]); must lie in [1e-20, 1e20] (the kernel adds the
+ *           bias through the tensor core as dt / scale), else DMA_ERR_INVALID_ARG.
  *   out     [B, L, Hq, d] bf16 (written; rows i >= len_b are computed with the same rule).
  */
 DMA_API dma_status_t dma_forward_prefill(const void* q, const void* k, const void* v, const float* W_dt, const float* A,

@@ -79,6 +79,10 @@ def test_argument_errors_are_reported_before_any_device_work(lib):
     assert lib.dma_forward_prefill(*a) == 2                     # DMA_ERR_UNSUPPORTED
     a = list(args); a[12] = float("nan")
     assert lib.dma_forward_prefill(*a) == 1
+    a = list(args); a[12] = 0.0
+    assert lib.dma_forward_prefill(*a) == 1                     # the prefill scale must be positive
+    a = list(args); a[12] = -0.125
+    assert lib.dma_forward_prefill(*a) == 1
     a = list(args); a[3] = None; a[4] = None
     assert lib.dma_forward_prefill(*a) == 1                     # neither W/A nor dt_in
     lib.dma_build_mask.restype = ctypes.c_int

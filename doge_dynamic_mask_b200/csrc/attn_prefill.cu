@@ -51,6 +51,9 @@ constexpr int kThreads = 352;   // 11 warps: K producer, MMA/TMEM, V producer, 2
 // 168 per thread is the most one CTA per SM can have)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+// every kPolyEvery-th pair of probabilities in a row is computed on the FMA pipe
+// (exp2_poly_x2), the rest on the MUFU
+constexpr int kPolyEvery = 4;
 constexpr int kXBytes = kKeyTile * 32;       // 128 rows x 16 bf16 extra K columns (bias / ones)
 
 template <int D>
@@ -123,6 +126,78 @@ __device__ __forceinline__ uint4 bias_columns(float c) {
   return make_uint4(hi | (mid << 16), lo, 0u, 0u);
 }
 
+// 2^x for two values at once on the FMA pipe, x <= 8 (the lazy rescale lets x
+// exceed 0 by up to its threshold).  x = n + f with n = round(x) and f in
+// [-1/2, 1/2]: 2^f comes from a cubic fitted to 2^f over that interval
+// (relative error below 7.5e-5, far under the bf16 rounding P goes through
+// next), and n is added straight into the exponent field.  Inputs are clamped
+// at -126 so the exponent field never underflows (masked keys, x = -inf, give
+// 2^-126 or less instead of 0: negligible next to the row maximum's weight 1).
+// Used for a fixed share of each row's probabilities, so that the
+// exponentials are split between this path and the MUFU ex2 unit.
+__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& p0, float& p1) {
+  const unsigned long long xa = f32x2(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const unsigned long long magic = f32x2(12582912.0f, 12582912.0f);   // 1.5 * 2^23
+  const unsigned long long t = add_f32x2(xa, magic);   // round(x) in the low mantissa bits
+  const unsigned long long f = sub_f32x2(xa, sub_f32x2(t, magic));
+  unsigned long long q = fma_f32x2(f, f32x2(0.0551716573536396f, 0.0551716573536396f),
+                                   f32x2(0.2426111400127411f, 0.2426111400127411f));
+  q = fma_f32x2(q, f, f32x2(0.6932609677314758f, 0.6932609677314758f));
+  q = fma_f32x2(q, f, f32x2(0.9999280571937561f, 0.9999280571937561f));
+  float q0, q1, t0, t1;
+  f32x2_split(q, q0, q1);
+  f32x2_split(t, t0, t1);
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
+// Tensor-memory columns: S_h at h * 128, O_h at 256 + h * D and, at d = 64,
+// P_h at 384 + h * 64 (otherwise P_h is written over S_h).
+//
+// S_h = Q_h K^T (+ dt/scale through the extra K=16 block) for the NH heads
+// h0 .. h0+NH-1 from K stage descriptors k_lo / kx_lo.  With two heads their
+// K steps alternate, so consecutive MMAs write different accumulators.
+template <int D, int NH>
+__device__ __forceinline__ void issue_qk(uint32_t tmem, int h0, uint32_t q_lo, uint32_t k_lo, uint32_t qx_lo,
+                                         uint32_t kx_lo, uint32_t idesc) {
+  constexpr uint32_t kQStep = (kRowTile * D * 2) >> 4;   // one head's Q tile, in 16-byte units
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = static_cast<uint32_t>(((kk / 4) * (kKeyTile * 128) + (kk % 4) * 32) >> 4);
+#pragma unroll
+    for (int i = 0; i < NH; ++i) {
+      const uint32_t h = static_cast<uint32_t>(h0 + i);
+      if (kk == 0)
+        umma_ss_w<0, kDescHiSw128, kDescHiSw128>(tmem + h * 128, q_lo + h * kQStep, k_lo, idesc);
+      else
+        umma_ss_w<1, kDescHiSw128, kDescHiSw128>(tmem + h * 128, q_lo + h * kQStep + off, k_lo + off, idesc);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < NH; ++i) {
+    const uint32_t h = static_cast<uint32_t>(h0 + i);
+    umma_ss_w<1, kDescHiPlain, kDescHiPlain>(tmem + h * 128, qx_lo + h * (kXBytes >> 4), kx_lo, idesc);
+  }
+}
+
+// O_h += P_h V for the NH heads h0 .. h0+NH-1 from V stage descriptor v_lo, K
+// steps alternating between heads.
+template <int D, int NH, bool SEP_P>
+__device__ __forceinline__ void issue_pv(uint32_t tmem, int h0, uint32_t v_lo, uint32_t idesc, bool first) {
+#pragma unroll
+  for (int kk = 0; kk < kKeyTile / 16; ++kk) {
+#pragma unroll
+    for (int i = 0; i < NH; ++i) {
+      const uint32_t h = static_cast<uint32_t>(h0 + i);
+      const uint32_t dO = tmem + 256 + h * D;
+      const uint32_t tp = (SEP_P ? tmem + 384 + h * 64 : tmem + h * 128) + kk * 8;
+      const uint32_t b = v_lo + static_cast<uint32_t>((kk * 2048) >> 4);
+      if (kk == 0 && first) umma_ts_w<0, kDescHiSw128>(dO, tp, b, idesc);
+      else umma_ts_w<1, kDescHiSw128>(dO, tp, b, idesc);
+    }
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
@@ -191,8 +266,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < C::kMetaSlots; ++s) mbar_init(bars.meta_full + s, 1);
     for (int h = 0; h < 2; ++h) {
       mbar_init(bars.s_full + h, 1);
-      mbar_init(bars.s_free + h, kRowTile);
-      mbar_init(bars.p_ready + h, kRowTile);
+      // the lockstep (separate-P) layout uses index 0 for both heads
+      mbar_init(bars.s_free + h, C::kSepP ? nh * kRowTile : kRowTile);
+      mbar_init(bars.p_ready + h, C::kSepP ? nh * kRowTile : kRowTile);
       mbar_init(bars.o_done + h, 1);
     }
     mbar_init(bars.fin, 1);
@@ -342,91 +418,90 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_qk = make_idesc_bf16(128, 128, false, false);
       const uint32_t idesc_pv = make_idesc_bf16(128, D, false, true);
-      const uint32_t q_addr = smem_u32(sQ), qx_addr = smem_u32(sQx), k_addr = smem_u32(sK),
-                     kx_addr = smem_u32(sKx), v_addr = smem_u32(sV);
+      // descriptor low words of every operand base (the high words are constants)
+      const uint32_t q_lo = desc_lo(smem_u32(sQ), 16), k_lo = desc_lo(smem_u32(sK), 16),
+                     v_lo = desc_lo(smem_u32(sV), C::kSlabBytes), qx_lo = desc_lo(smem_u32(sQx), 128),
+                     kx_lo = desc_lo(smem_u32(sKx), 128);
+      constexpr uint32_t kKVStep = C::kKVBytes >> 4, kXStep = kXBytes >> 4;
       bool ok = mbar_wait_hot(bars.q_full, 0, err, kDevErrTimeoutBase + 4);
-      // Descriptor bases, computed once: a stage, a head or a K step only moves
-      // the 14-bit start-address field (16-byte units; shared memory < 256 KB),
-      // so every MMA below costs a couple of integer adds to issue.
-      const uint64_t qd0 = make_sw128_desc(q_addr, 16, 1024);
-      const uint64_t kd0 = make_sw128_desc(k_addr, 16, 1024);
-      const uint64_t vd0 = make_sw128_desc(v_addr, C::kSlabBytes, 1024);
-      const uint64_t qxd0 = make_noswizzle_desc(qx_addr, 128, 256);
-      const uint64_t kxd0 = make_noswizzle_desc(kx_addr, 128, 256);
-      auto issue_qk = [&](int h, int s) {
-        const uint64_t qa = qd0 + static_cast<uint64_t>(h * (C::kQBytes >> 4));
-        const uint64_t kb = kd0 + static_cast<uint64_t>(s * (C::kKVBytes >> 4));
-        const uint32_t dS = tmem + h * 128;
-        umma_ss_c<0>(dS, qa, kb, idesc_qk);
-#pragma unroll
-        for (int kk = 1; kk < D / 16; ++kk) {
-          const uint64_t off = static_cast<uint64_t>(((kk / 4) * C::kSlabBytes + (kk % 4) * 32) >> 4);
-          umma_ss_c<1>(dS, qa + off, kb + off, idesc_qk);
-        }
-        // + dt/scale through the extra K=16 block (ones x bias columns)
-        umma_ss_c<1>(dS, qxd0 + static_cast<uint64_t>(h * (kXBytes >> 4)),
-                     kxd0 + static_cast<uint64_t>(s * (kXBytes >> 4)), idesc_qk);
-        umma_commit(bars.s_full + h);
-      };
-      auto issue_pv = [&](int h, int s, bool first) {
-        const uint64_t vb = vd0 + static_cast<uint64_t>(s * (C::kKVBytes >> 4));
-        const uint32_t dO = tmem + 256 + h * D;
-        const uint32_t tp = C::kSepP ? tmem + 384 + h * 64 : tmem + h * 128;
-        if (first) umma_ts_c<0>(dO, tp, vb, idesc_pv); else umma_ts_c<1>(dO, tp, vb, idesc_pv);
-#pragma unroll
-        for (int kk = 1; kk < kKeyTile / 16; ++kk)
-          umma_ts_c<1>(dO, tp + kk * 8, vb + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv);
-        umma_commit(bars.o_done + h);
-      };
-      // Event-driven issue: poll every pending barrier and issue whichever MMA
-      // is ready, so one head never waits on the other's progress (the tensor
-      // core still executes in issue order).
-      //   QK_h(j): needs K(j) landed and S_h free (separate P: S_h(j-1) read by
-      //            the softmax; P over S: PV_h(j-1) issued before it)
-      //   PV_h(j): needs P_h(j) written and V(j) landed
-      // A K stage is released once both heads' QK of it are issued, a V stage
-      // once both PVs are.
-      int next_qk[2] = {0, 0}, next_pv[2] = {0, 0};
-      long long t_last = clock64();   // last time an MMA was issued
-      while (ok) {
-        bool all_done = true, progressed = false;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (h >= nh) continue;
-          const int jq = next_qk[h];
-          if (jq < n_kt) {
-            all_done = false;
-            const bool s_ready = jq == 0 || (C::kSepP ? mbar_test(bars.s_free + h, (jq - 1) & 1)
-                                                      : next_pv[h] >= jq);
-            if (s_ready && mbar_test(bars.k_full + jq % C::kStages, (jq / C::kStages) & 1)) {
-              tc_fence_after();
-              issue_qk(h, jq % C::kStages);
-              next_qk[h] = jq + 1;
-              progressed = true;
-              if (next_qk[0] >= jq + 1 && (nh < 2 || next_qk[1] >= jq + 1)) umma_commit(bars.k_empty + jq % C::kStages);
-            }
-          }
-          const int jp = next_pv[h];
-          if (jp < n_kt) {
-            all_done = false;
-            if (jp < next_qk[h] && mbar_test(bars.p_ready + h, jp & 1) &&
-                mbar_test(bars.v_full + jp % C::kStages, (jp / C::kStages) & 1)) {
-              tc_fence_after();
-              issue_pv(h, jp % C::kStages, jp == 0);
-              next_pv[h] = jp + 1;
-              progressed = true;
-              if (next_pv[0] >= jp + 1 && (nh < 2 || next_pv[1] >= jp + 1)) umma_commit(bars.v_empty + jp % C::kStages);
-            }
+      // Issue-wait: polls the barrier, gives up on a CTA abort or after the cycle limit.
+      auto wait = [&](uint64_t* b, uint32_t parity, uint32_t site) -> bool {
+        if (mbar_try_wait(b, parity)) return true;
+        const long long t0 = clock64();
+        while (true) {
+          if (mbar_try_wait(b, parity)) return true;
+          if (aborted(abort_flag)) return false;
+          if (clock64() - t0 > kWaitLimitCycles) {
+            raise_error(err, kDevErrTimeoutBase + site);
+            return false;
           }
         }
-        if (all_done) break;
-        if (progressed) {
-          t_last = clock64();
+      };
+      if (ok && n_kt > 0) ok = wait(bars.k_full, 0, 1);
+      if (ok && n_kt > 0) {
+        tc_fence_after();
+        if constexpr (C::kSepP) {
+          if (nh == 2) issue_qk<D, 2>(tmem, 0, q_lo, k_lo, qx_lo, kx_lo, idesc_qk);
+          else issue_qk<D, 1>(tmem, 0, q_lo, k_lo, qx_lo, kx_lo, idesc_qk);
+          umma_commit(bars.s_full);
         } else {
-          if (aborted(abort_flag) || clock64() - t_last > kWaitLimitCycles) {
-            raise_error(err, kDevErrTimeoutBase + 16);
-            ok = false;
+          for (int h = 0; h < nh; ++h) {
+            issue_qk<D, 1>(tmem, h, q_lo, k_lo, qx_lo, kx_lo, idesc_qk);
+            umma_commit(bars.s_full + h);
           }
+        }
+        umma_commit(bars.k_empty);
+      }
+      if constexpr (C::kSepP) {
+        // Both heads in lockstep (one S/P/O barrier set for the pair).  The
+        // softmax releases S right after reading it, so QK(j+1) goes in as soon
+        // as that happens and runs during the softmax of tile j; PV(j) follows
+        // once both heads' P(j) are written.  Queue: ... PV(j-1), QK(j+1), PV(j) ...
+        for (int j = 0; ok && j < n_kt; ++j) {
+          const int s = j % C::kStages;
+          if (j + 1 < n_kt) {
+            const int s1 = (j + 1) % C::kStages;
+            ok = wait(bars.s_free, j & 1, 5) && wait(bars.k_full + s1, ((j + 1) / C::kStages) & 1, 6);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t kl = k_lo + s1 * kKVStep, kxl = kx_lo + s1 * kXStep;
+            if (nh == 2) issue_qk<D, 2>(tmem, 0, q_lo, kl, qx_lo, kxl, idesc_qk);
+            else issue_qk<D, 1>(tmem, 0, q_lo, kl, qx_lo, kxl, idesc_qk);
+            umma_commit(bars.s_full);
+            umma_commit(bars.k_empty + s1);
+          }
+          ok = wait(bars.p_ready, j & 1, 7) && wait(bars.v_full + s, (j / C::kStages) & 1, 8);
+          if (!ok) break;
+          tc_fence_after();
+          if (nh == 2) issue_pv<D, 2, true>(tmem, 0, v_lo + s * kKVStep, idesc_pv, j == 0);
+          else issue_pv<D, 1, true>(tmem, 0, v_lo + s * kKVStep, idesc_pv, j == 0);
+          umma_commit(bars.o_done);
+          umma_commit(bars.v_empty + s);
+        }
+      } else {
+        // P is written over S, so QK_h(j+1) can only follow PV_h(j).  Fixed
+        // ping-pong order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1): while one
+        // head's softmax runs, the tensor core works through the other head's
+        // PV and next QK.
+        for (int j = 0; ok && j < n_kt; ++j) {
+          const int s = j % C::kStages, s1 = (j + 1) % C::kStages;
+          for (int h = 0; ok && h < nh; ++h) {
+            ok = wait(bars.p_ready + h, j & 1, 7) && (h > 0 || wait(bars.v_full + s, (j / C::kStages) & 1, 8));
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv<D, 1, false>(tmem, h, v_lo + s * kKVStep, idesc_pv, j == 0);
+            umma_commit(bars.o_done + h);
+            if (j + 1 < n_kt) {
+              ok = h > 0 || wait(bars.k_full + s1, ((j + 1) / C::kStages) & 1, 6);
+              if (!ok) break;
+              tc_fence_after();
+              issue_qk<D, 1>(tmem, h, q_lo, k_lo + s1 * kKVStep, qx_lo, kx_lo + s1 * kXStep, idesc_qk);
+              umma_commit(bars.s_full + h);
+            }
+          }
+          if (!ok) break;
+          umma_commit(bars.v_empty + s);
+          if (j + 1 < n_kt) umma_commit(bars.k_empty + s1);
         }
       }
       if (!ok) *abort_flag = 1;
@@ -447,9 +522,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m = -INFINITY, l = 0.0f;
       bool ok = true;
       const unsigned long long scale2 = f32x2(scale_log2, scale_log2);
+      // barrier index: the lockstep layout (separate P) has one set for the pair
+      const int hb = C::kSepP ? 0 : h;
       for (int j = 0; j < n_kt; ++j) {
         const int ms_slot = j % C::kMetaSlots;
-        ok = mbar_wait(bars.s_full + h, j & 1, err, kDevErrTimeoutBase + 10);
+        ok = mbar_wait(bars.s_full + hb, j & 1, err, kDevErrTimeoutBase + 10);
         // the tile's row-interval table (published by the K producer)
         if (ok) ok = mbar_wait(bars.meta_full + ms_slot, (j / C::kMetaSlots) & 1, err, kDevErrTimeoutBase + 13);
         if (!ok || aborted(abort_flag)) {
@@ -465,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         if constexpr (C::kSepP) {
           tc_fence_before();
-          mbar_arrive(bars.s_free + h);   // S may be overwritten by the next Q K^T
+          mbar_arrive(bars.s_free);   // S may be overwritten by the next Q K^T
         }
         if (!((j + 1) * kKeyTile <= n_full || !row_valid)) {
           // key tile not kept by every row: drop keys outside this row's interval
@@ -501,36 +578,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float nm = m == -INFINITY ? 0.0f : -m;
         const unsigned long long nm2 = f32x2(nm, nm);
+        unsigned long long sa = 0ull, sb = 0ull;   // two packed partial sums
+        // p = 2^(x * scale * log2e - m) for two keys, packed as bf16x2
+        auto p_pair = [&](int k) -> uint32_t {
+          const unsigned long long x2 =
+              fma_f32x2(f32x2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), scale2, nm2);
+          float x0, x1, p0, p1;
+          f32x2_split(x2, x0, x1);
+          if (((k >> 1) % kPolyEvery) == kPolyEvery - 1) {
+            exp2_poly_x2(x0, x1, p0, p1);
+          } else {
+            p0 = fast_exp2(x0);
+            p1 = fast_exp2(x1);
+          }
+          if ((k >> 1) & 1) sb = add_f32x2(sb, f32x2(p0, p1)); else sa = add_f32x2(sa, f32x2(p0, p1));
+          return pack_bf16x2(p0, p1);
+        };
         if constexpr (C::kSepP) {
-          // P's columns and O are free once PV of the previous tile is done
+          // all of P in registers first: only its store has to wait for PV of
+          // the previous tile (which reads P's columns)
+          uint32_t pk[64];
+#pragma unroll
+          for (int c = 0; c < 64; ++c) pk[c] = p_pair(2 * c);
           if (j > 0) {
-            ok = mbar_wait(bars.o_done + h, (j - 1) & 1, err, kDevErrTimeoutBase + 11);
+            ok = mbar_wait(bars.o_done, (j - 1) & 1, err, kDevErrTimeoutBase + 11);
             if (!ok) {
               *abort_flag = 1;
               break;
             }
             tc_fence_after();
           }
-        }
-        const uint32_t tP = C::kSepP ? tmem + lane_base + 384 + h * 64 : tS;
-        unsigned long long sa = 0ull, sb = 0ull;   // two packed partial sums
-        // P in two halves of 64 keys (32 packed columns each)
+          const uint32_t tP = tmem + lane_base + 384 + h * 64;
+          DMA_TMEM_ST32(tP, pk);
+          DMA_TMEM_ST32(tP + 32, (pk + 32));
+        } else {
+          // P over S, in two halves of 64 keys (32 packed columns each)
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
+          for (int half = 0; half < 2; ++half) {
+            uint32_t pk[32];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int k = 64 * half + 2 * c;
-            const unsigned long long x2 =
-                fma_f32x2(f32x2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), scale2, nm2);
-            float x0, x1;
-            f32x2_split(x2, x0, x1);
-            const float p0 = fast_exp2(x0);
-            const float p1 = fast_exp2(x1);
-            if (c & 1) sb = add_f32x2(sb, f32x2(p0, p1)); else sa = add_f32x2(sa, f32x2(p0, p1));
-            pk[c] = pack_bf16x2(p0, p1);
+            for (int c = 0; c < 32; ++c) pk[c] = p_pair(64 * half + 2 * c);
+            DMA_TMEM_ST32(tS + 32 * half, pk);
           }
-          DMA_TMEM_ST32(tP + 32 * half, pk);
+          // consume every o_done phase in order (PV of the previous tile), so
+          // the parity of the epilogue's wait is never ambiguous
+          if (j > 0) {
+            ok = mbar_wait(bars.o_done + h, (j - 1) & 1, err, kDevErrTimeoutBase + 11);
+            if (!ok) {
+              *abort_flag = 1;
+              tmem_wait_st();
+              break;
+            }
+            tc_fence_after();
+          }
         }
         {
           float a0, a1, b0, b1;
@@ -538,36 +638,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           f32x2_split(sb, b0, b1);
           l += (a0 + a1) + (b0 + b1);
         }
-        if (j > 0) {
-          // consume every o_done phase in order (PV of the previous tile), so
-          // the parity of the epilogue's wait is never ambiguous
-          if constexpr (!C::kSepP) ok = mbar_wait(bars.o_done + h, (j - 1) & 1, err, kDevErrTimeoutBase + 11);
-          if (!ok) {
-            *abort_flag = 1;
-            tmem_wait_st();
-            break;
-          }
-          // rescale O (only warps where some row's max moved far enough)
-          if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
-            tc_fence_after();
+        // rescale O (only warps where some row's max moved far enough); PV of
+        // the previous tile is complete (waited above)
+        if (j > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-              uint32_t o[32];
-              DMA_TMEM_LD32(tO + c0, o);
-              tmem_wait_ld();
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o[32];
+            DMA_TMEM_LD32(tO + c0, o);
+            tmem_wait_ld();
 #pragma unroll
-              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-              DMA_TMEM_ST32(tO + c0, o);
-            }
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            DMA_TMEM_ST32(tO + c0, o);
           }
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bars.p_ready + h);
+        mbar_arrive(bars.p_ready + hb);
       }
       // epilogue
       if (ok && !aborted(abort_flag) && n_kt > 0) {
-        ok = mbar_wait(bars.o_done + h, (n_kt - 1) & 1, err, kDevErrTimeoutBase + 12);
+        ok = mbar_wait(bars.o_done + hb, (n_kt - 1) & 1, err, kDevErrTimeoutBase + 12);
         if (ok) {
           tc_fence_after();
           const float inv = 1.0f / l;

@@ -192,6 +192,37 @@ __device__ __forceinline__ void umma_ts_c(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
+// Descriptors split in two 32-bit words: the high word (stride byte offset,
+// version, layout) is a compile-time constant per operand kind, and only the
+// low word (start address >> 4, leading byte offset) changes from one MMA to
+// the next, so an issuing thread keeps one 32-bit register per operand base
+// and advances it with a single add.
+__host__ __device__ constexpr uint32_t desc_hi(uint32_t sbo_bytes, uint32_t layout) {
+  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (layout << 29);
+}
+__device__ __forceinline__ uint32_t desc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+constexpr uint32_t kDescHiSw128 = desc_hi(1024, 2);     // 128-byte swizzle, 8-row groups 1024 B apart
+constexpr uint32_t kDescHiPlain = desc_hi(256, 0);      // no swizzle, 8-row groups 256 B apart
+
+// D[tmem] (+)= A[smem] * B[smem] from descriptor low words (high words AHI, BHI).
+template <int ACC, uint32_t AHI, uint32_t BHI>
+__device__ __forceinline__ void umma_ss_w(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\tmov.b64 ad, {%1, %5};\n\tmov.b64 bd, {%2, %6};\n\t"
+      "setp.ne.b32 p, %4, 0;\n\ttcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(idesc), "n"(ACC), "r"(AHI), "r"(BHI));
+}
+// D[tmem] (+)= A[tmem] * B[smem] from the B descriptor's low word (high word BHI).
+template <int ACC, uint32_t BHI>
+__device__ __forceinline__ void umma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 bd;\n\tmov.b64 bd, {%2, %5};\n\t"
+      "setp.ne.b32 p, %4, 0;\n\ttcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(idesc), "n"(ACC), "r"(BHI));
+}
+
 // Arrive on an mbarrier once every previously issued tcgen05.mma of this thread has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -298,6 +329,11 @@ __device__ __forceinline__ unsigned long long fma_f32x2(unsigned long long a, un
                                                         unsigned long long c) {
   unsigned long long d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long sub_f32x2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
 __device__ __forceinline__ unsigned long long add_f32x2(unsigned long long a, unsigned long long b) {

@@ -72,7 +72,7 @@ struct Cfg {
   static constexpr int kOffV = kOffKx + kStages * kXBytes;
   static constexpr int kOffMeta = kOffV + kStages * kKVBytes;
   static constexpr int kOffBar = kOffMeta + kMetaSlots * kMetaBytes;
-  static constexpr int kNumBars = 1 + 4 * kStages + kMetaSlots + 8 + 1;
+  static constexpr int kNumBars = 2 + 4 * kStages + kMetaSlots + 8 + 1;
   // d = 64 leaves TMEM room for P in its own columns (S 2x128, O 2x64, P 2x64):
   // the softmax releases S as soon as it has read it, and the next S = Q K^T
   // overlaps the current softmax.  At d = 128 (O 2x128) P is written over S.
@@ -92,6 +92,7 @@ struct Cfg {
 // one phase behind.
 struct Bars {
   uint64_t* q_full;
+  uint64_t* q_empty;    // the CTA's Q tile may be refilled (all Q K^T of the item done)
   uint64_t* k_full;     // [stages]
   uint64_t* v_full;     // [stages]
   uint64_t* k_empty;    // [stages]
@@ -198,6 +199,32 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem, int h0, uint32_t v_lo, u
   }
 }
 
+// Work item (heavy row tiles first): pair of query heads, kv head g, batch b, row tile t.
+struct Item {
+  int pair, g, b, t;
+};
+__device__ __forceinline__ Item decode_item(int w, int npairs, int Hkv, int B, int n_rt) {
+  Item it;
+  it.pair = w % npairs;
+  w /= npairs;
+  it.g = w % Hkv;
+  w /= Hkv;
+  it.b = w % B;
+  it.t = n_rt - 1 - w / B;
+  return it;
+}
+// The i-th work item of this CTA: rounds of gridDim.x items, taken forwards in
+// even rounds and backwards in odd ones, so every CTA gets a similar mix of
+// heavy and light row tiles.
+__device__ __forceinline__ int item_of(int i) {
+  const int P = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  return i * P + ((i & 1) ? P - 1 - c : c);
+}
+
+// Persistent kernel: one CTA per SM walks its share of the work items; every
+// role counts key tiles across items, so barrier phases and ring slots carry on
+// from one item to the next and the next item's Q, K, V and first S = Q K^T
+// are in flight while the softmax warps finish the current item's output.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
@@ -213,6 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   {
     uint64_t* p = bar;
     bars.q_full = p; p += 1;
+    bars.q_empty = p; p += 1;
     bars.k_full = p; p += C::kStages;
     bars.v_full = p; p += C::kStages;
     bars.k_empty = p; p += C::kStages;
@@ -227,25 +255,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
 
-  // ---- work item: heavy row tiles first ------------------------------------
   const int n_rt = plan.n_row_tiles;
   const int nrep = Hq / Hkv;
   const int npairs = (nrep + 1) / 2;
-  int id = blockIdx.x;
-  const int pair = id % npairs;
-  id /= npairs;
-  const int g = id % Hkv;
-  id /= Hkv;
-  const int b = id % B;
-  const int t = n_rt - 1 - id / B;
-  const int nh = min(2, nrep - 2 * pair);            // query heads in this CTA
-  const int h0 = g * nrep + 2 * pair;                // first query head
-  const int r0 = t * kRowTile;
-  const int nrows = min(kRowTile, L - r0);
-  const size_t tile = (static_cast<size_t>(b) * Hkv + g) * n_rt + t;
-  const int2 cnt = plan.counts[tile];
-  const int n_full = cnt.x, n_total = cnt.y;
-  const int n_kt = (n_total + kKeyTile - 1) / kKeyTile;
+  const int n_items = n_rt * B * Hkv * npairs;
+  // Softmax head slots taking part in the lockstep (separate-P) barriers: when
+  // a pair has a single head (odd nrep), the other slot's warps still arrive
+  // on them without doing any work, so their counts never change.
+  const int hw = nrep >= 2 ? 2 : 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned char* sQ = smem + C::kOffQ;
@@ -257,6 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bars.q_full, 1);
+    mbar_init(bars.q_empty, 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(bars.k_full + s, 1);
       mbar_init(bars.v_full + s, 1);
@@ -267,8 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int h = 0; h < 2; ++h) {
       mbar_init(bars.s_full + h, 1);
       // the lockstep (separate-P) layout uses index 0 for both heads
-      mbar_init(bars.s_free + h, C::kSepP ? nh * kRowTile : kRowTile);
-      mbar_init(bars.p_ready + h, C::kSepP ? nh * kRowTile : kRowTile);
+      mbar_init(bars.s_free + h, C::kSepP ? hw * kRowTile : kRowTile);
+      mbar_init(bars.p_ready + h, C::kSepP ? hw * kRowTile : kRowTile);
       mbar_init(bars.o_done + h, 1);
     }
     mbar_init(bars.fin, 1);
@@ -299,118 +317,162 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int32_t* idx_t = plan.idx + tile * plan.cap;
-  const int32_t* kbase_t = plan.kbase + tile * (plan.cap / kKeyTile);
-  const float* bias_t = plan.bias + tile * plan.cap;
-  const uint32_t* span_t = plan.span + tile * plan.cap;
-  const int base_row = b * L;
+
+  // work item i of this CTA: false when there is none left
+  struct ItemInfo {
+    Item it;
+    int nh, n_kt, n_full;
+    size_t tile;
+  };
+  auto item_info = [&](int i, ItemInfo& x) -> bool {
+    const int w = item_of(i);
+    if (w >= n_items) return false;
+    x.it = decode_item(w, npairs, Hkv, B, n_rt);
+    x.nh = min(2, nrep - 2 * x.it.pair);
+    x.tile = (static_cast<size_t>(x.it.b) * Hkv + x.it.g) * n_rt + x.it.t;
+    const int2 cnt = plan.counts[x.tile];
+    x.n_full = cnt.x;
+    x.n_kt = (cnt.y + kKeyTile - 1) / kKeyTile;
+    return true;
+  };
 
   if (warp == 0) {
     // ======================= K producer =====================================
-    int issued = 0;
-    if (lane == 0) mbar_arrive_expect_tx(bars.q_full, nh * C::kQBytes);
-    __syncwarp();
-    if (lane < nh * C::kSlabs) {
-      const int h = lane / C::kSlabs, sl = lane % C::kSlabs;
-      tma_load_3d(sQ + h * C::kQBytes + sl * C::kSlabBytes, &tmap_q, bars.q_full, sl * 64, h0 + h,
-                  base_row + r0);
-    }
-    for (int j = 0; j < n_kt; ++j) {
-      const int s = j % C::kStages;
-      const int u = j / C::kStages;
-      const int ms_slot = j % C::kMetaSlots;
-      if (j >= C::kStages && !mbar_wait(bars.k_empty + s, (u - 1) & 1, err, kDevErrTimeoutBase + 1)) {
+    int gk = 0, nq = 0;   // K tiles and Q tiles issued so far
+    bool stop = false;
+    ItemInfo x;
+    for (int i = 0; !stop && item_info(i, x); ++i) {
+      if (x.n_kt == 0) continue;
+      const int g = x.it.g, base_row = x.it.b * L;
+      const int h0 = g * nrep + 2 * x.it.pair;
+      // Q: the previous item's Q K^T must be complete
+      if (nq > 0 && !mbar_wait(bars.q_empty, (nq - 1) & 1, err, kDevErrTimeoutBase + 15)) {
         *abort_flag = 1;
         break;
       }
       if (aborted(abort_flag)) break;
-      const int e = j * kKeyTile + lane * 4;
-      const int kb0 = kbase_t[j];
-      {
-        const float4 bi = *reinterpret_cast<const float4*>(bias_t + e);
-        const uint4 sp = *reinterpret_cast<const uint4*>(span_t + e);
-        *reinterpret_cast<uint4*>(sMeta + ms_slot * C::kMetaBytes + lane * 16) = sp;
-        const float bv[4] = {bi.x, bi.y, bi.z, bi.w};
+      if (lane == 0) mbar_arrive_expect_tx(bars.q_full, x.nh * C::kQBytes);
+      __syncwarp();
+      if (lane < x.nh * C::kSlabs) {
+        const int h = lane / C::kSlabs, sl = lane % C::kSlabs;
+        tma_load_3d(sQ + h * C::kQBytes + sl * C::kSlabBytes, &tmap_q, bars.q_full, sl * 64, h0 + h,
+                    base_row + x.it.t * kRowTile);
+      }
+      ++nq;
+      const int32_t* idx_t = plan.idx + x.tile * plan.cap;
+      const int32_t* kbase_t = plan.kbase + x.tile * (plan.cap / kKeyTile);
+      const float* bias_t = plan.bias + x.tile * plan.cap;
+      const uint32_t* span_t = plan.span + x.tile * plan.cap;
+      for (int j = 0; j < x.n_kt; ++j, ++gk) {
+        const int s = gk % C::kStages;
+        const int u = gk / C::kStages;
+        const int ms_slot = gk % C::kMetaSlots;
+        if (gk >= C::kStages && !mbar_wait(bars.k_empty + s, (u - 1) & 1, err, kDevErrTimeoutBase + 1)) {
+          *abort_flag = 1;
+          stop = true;
+          break;
+        }
+        if (aborted(abort_flag)) {
+          stop = true;
+          break;
+        }
+        const int e = j * kKeyTile + lane * 4;
+        const int kb0 = kbase_t[j];
+        {
+          const float4 bi = *reinterpret_cast<const float4*>(bias_t + e);
+          const uint4 sp = *reinterpret_cast<const uint4*>(span_t + e);
+          *reinterpret_cast<uint4*>(sMeta + ms_slot * C::kMetaBytes + lane * 16) = sp;
+          const float bv[4] = {bi.x, bi.y, bi.z, bi.w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          *reinterpret_cast<uint4*>(sKx + s * kXBytes + xoff(lane * 4 + q, 0)) = bias_columns(bv[q] * inv_scale);
-      }
-      fence_proxy_async_smem();   // the bias block is read by the tensor core
-      int4 ix = make_int4(0, 0, 0, 0);
-      if (kb0 < 0) {
-        ix = *reinterpret_cast<const int4*>(idx_t + e);
-        ix.x = (base_row + ix.x) * Hkv + g;
-        ix.y = (base_row + ix.y) * Hkv + g;
-        ix.z = (base_row + ix.z) * Hkv + g;
-        ix.w = (base_row + ix.w) * Hkv + g;
-      }
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bars.meta_full + ms_slot);
-        mbar_arrive_expect_tx(bars.k_full + s, C::kKVBytes);
-      }
-      __syncwarp();
-      if (kb0 >= 0) {
-        // one ascending run of keys: a 128-row box per 64-column slab
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(sKx + s * kXBytes + xoff(lane * 4 + q, 0)) = bias_columns(bv[q] * inv_scale);
+        }
+        fence_proxy_async_smem();   // the bias block is read by the tensor core
+        int4 ix = make_int4(0, 0, 0, 0);
+        if (kb0 < 0) {
+          ix = *reinterpret_cast<const int4*>(idx_t + e);
+          ix.x = (base_row + ix.x) * Hkv + g;
+          ix.y = (base_row + ix.y) * Hkv + g;
+          ix.z = (base_row + ix.z) * Hkv + g;
+          ix.w = (base_row + ix.w) * Hkv + g;
+        }
+        __syncwarp();
         if (lane == 0) {
+          mbar_arrive(bars.meta_full + ms_slot);
+          mbar_arrive_expect_tx(bars.k_full + s, C::kKVBytes);
+        }
+        __syncwarp();
+        if (kb0 >= 0) {
+          // one ascending run of keys: a 128-row box per 64-column slab
+          if (lane == 0) {
+#pragma unroll
+            for (int sl = 0; sl < C::kSlabs; ++sl)
+              tma_load_3d(sK + s * C::kKVBytes + sl * C::kSlabBytes, &tmap_k3, bars.k_full + s, sl * 64, g,
+                          base_row + kb0);
+          }
+        } else {
 #pragma unroll
           for (int sl = 0; sl < C::kSlabs; ++sl)
-            tma_load_3d(sK + s * C::kKVBytes + sl * C::kSlabBytes, &tmap_k3, bars.k_full + s, sl * 64, g,
-                        base_row + kb0);
+            tma_gather4(sK + s * C::kKVBytes + sl * C::kSlabBytes + lane * 512, &tmap_k, bars.k_full + s, sl * 64,
+                        ix.x, ix.y, ix.z, ix.w);
         }
-      } else {
-#pragma unroll
-        for (int sl = 0; sl < C::kSlabs; ++sl)
-          tma_gather4(sK + s * C::kKVBytes + sl * C::kSlabBytes + lane * 512, &tmap_k, bars.k_full + s, sl * 64,
-                      ix.x, ix.y, ix.z, ix.w);
       }
-      issued = j + 1;
     }
     // drain: every copy issued must have landed before the CTA can leave
     if (lane == 0) {
-      mbar_wait(bars.q_full, 0, err, kDevErrTimeoutBase + 2);
-      for (int j = issued - C::kStages < 0 ? 0 : issued - C::kStages; j < issued; ++j)
+      if (nq > 0) mbar_wait(bars.q_full, (nq - 1) & 1, err, kDevErrTimeoutBase + 2);
+      for (int j = gk - C::kStages < 0 ? 0 : gk - C::kStages; j < gk; ++j)
         mbar_wait(bars.k_full + j % C::kStages, (j / C::kStages) & 1, err, kDevErrTimeoutBase + 3);
     }
   } else if (warp == 2) {
     // ======================= V producer =====================================
-    int issued = 0;
-    for (int j = 0; j < n_kt; ++j) {
-      const int s = j % C::kStages;
-      const int u = j / C::kStages;
-      if (j >= C::kStages && !mbar_wait(bars.v_empty + s, (u - 1) & 1, err, kDevErrTimeoutBase + 14)) {
-        *abort_flag = 1;
-        break;
-      }
-      if (aborted(abort_flag)) break;
-      const int kb0 = kbase_t[j];
-      int4 ix = make_int4(0, 0, 0, 0);
-      if (kb0 < 0) {
-        ix = *reinterpret_cast<const int4*>(idx_t + j * kKeyTile + lane * 4);
-        ix.x = (base_row + ix.x) * Hkv + g;
-        ix.y = (base_row + ix.y) * Hkv + g;
-        ix.z = (base_row + ix.z) * Hkv + g;
-        ix.w = (base_row + ix.w) * Hkv + g;
-      }
-      if (lane == 0) mbar_arrive_expect_tx(bars.v_full + s, C::kKVBytes);
-      __syncwarp();
-      if (kb0 >= 0) {
-        if (lane == 0) {
+    int gv = 0;
+    bool stop = false;
+    ItemInfo x;
+    for (int i = 0; !stop && item_info(i, x); ++i) {
+      const int g = x.it.g, base_row = x.it.b * L;
+      const int32_t* idx_t = plan.idx + x.tile * plan.cap;
+      const int32_t* kbase_t = plan.kbase + x.tile * (plan.cap / kKeyTile);
+      for (int j = 0; j < x.n_kt; ++j, ++gv) {
+        const int s = gv % C::kStages;
+        const int u = gv / C::kStages;
+        if (gv >= C::kStages && !mbar_wait(bars.v_empty + s, (u - 1) & 1, err, kDevErrTimeoutBase + 14)) {
+          *abort_flag = 1;
+          stop = true;
+          break;
+        }
+        if (aborted(abort_flag)) {
+          stop = true;
+          break;
+        }
+        const int kb0 = kbase_t[j];
+        int4 ix = make_int4(0, 0, 0, 0);
+        if (kb0 < 0) {
+          ix = *reinterpret_cast<const int4*>(idx_t + j * kKeyTile + lane * 4);
+          ix.x = (base_row + ix.x) * Hkv + g;
+          ix.y = (base_row + ix.y) * Hkv + g;
+          ix.z = (base_row + ix.z) * Hkv + g;
+          ix.w = (base_row + ix.w) * Hkv + g;
+        }
+        if (lane == 0) mbar_arrive_expect_tx(bars.v_full + s, C::kKVBytes);
+        __syncwarp();
+        if (kb0 >= 0) {
+          if (lane == 0) {
+#pragma unroll
+            for (int sl = 0; sl < C::kSlabs; ++sl)
+              tma_load_3d(sV + s * C::kKVBytes + sl * C::kSlabBytes, &tmap_v3, bars.v_full + s, sl * 64, g,
+                          base_row + kb0);
+          }
+        } else {
 #pragma unroll
           for (int sl = 0; sl < C::kSlabs; ++sl)
-            tma_load_3d(sV + s * C::kKVBytes + sl * C::kSlabBytes, &tmap_v3, bars.v_full + s, sl * 64, g,
-                        base_row + kb0);
+            tma_gather4(sV + s * C::kKVBytes + sl * C::kSlabBytes + lane * 512, &tmap_v, bars.v_full + s, sl * 64,
+                        ix.x, ix.y, ix.z, ix.w);
         }
-      } else {
-#pragma unroll
-        for (int sl = 0; sl < C::kSlabs; ++sl)
-          tma_gather4(sV + s * C::kKVBytes + sl * C::kSlabBytes + lane * 512, &tmap_v, bars.v_full + s, sl * 64,
-                      ix.x, ix.y, ix.z, ix.w);
       }
-      issued = j + 1;
     }
     if (lane == 0) {
-      for (int j = issued - C::kStages < 0 ? 0 : issued - C::kStages; j < issued; ++j)
+      for (int j = gv - C::kStages < 0 ? 0 : gv - C::kStages; j < gv; ++j)
         mbar_wait(bars.v_full + j % C::kStages, (j / C::kStages) & 1, err, kDevErrTimeoutBase + 3);
     }
   } else if (warp == 1) {
@@ -423,7 +485,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                      v_lo = desc_lo(smem_u32(sV), C::kSlabBytes), qx_lo = desc_lo(smem_u32(sQx), 128),
                      kx_lo = desc_lo(smem_u32(sKx), 128);
       constexpr uint32_t kKVStep = C::kKVBytes >> 4, kXStep = kXBytes >> 4;
-      bool ok = mbar_wait_hot(bars.q_full, 0, err, kDevErrTimeoutBase + 4);
       // Issue-wait: polls the barrier, gives up on a CTA abort or after the cycle limit.
       auto wait = [&](uint64_t* b, uint32_t parity, uint32_t site) -> bool {
         if (mbar_try_wait(b, parity)) return true;
@@ -437,72 +498,99 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       };
-      if (ok && n_kt > 0) ok = wait(bars.k_full, 0, 1);
-      if (ok && n_kt > 0) {
-        tc_fence_after();
+      bool ok = true;
+      int g = 0, nq = 0, t1 = 0;   // key tiles so far (all items), items started, head-1 key tiles (d = 128)
+      ItemInfo x;
+      for (int i = 0; ok && item_info(i, x); ++i) {
+        const int n_kt = x.n_kt, nh = x.nh;
+        if (n_kt == 0) continue;
+        ok = wait(bars.q_full, nq & 1, 4);
+        ++nq;
+        if (!ok) break;
         if constexpr (C::kSepP) {
-          if (nh == 2) issue_qk<D, 2>(tmem, 0, q_lo, k_lo, qx_lo, kx_lo, idesc_qk);
-          else issue_qk<D, 1>(tmem, 0, q_lo, k_lo, qx_lo, kx_lo, idesc_qk);
-          umma_commit(bars.s_full);
-        } else {
-          for (int h = 0; h < nh; ++h) {
-            issue_qk<D, 1>(tmem, h, q_lo, k_lo, qx_lo, kx_lo, idesc_qk);
-            umma_commit(bars.s_full + h);
-          }
-        }
-        umma_commit(bars.k_empty);
-      }
-      if constexpr (C::kSepP) {
-        // Both heads in lockstep (one S/P/O barrier set for the pair).  The
-        // softmax releases S right after reading it, so QK(j+1) goes in as soon
-        // as that happens and runs during the softmax of tile j; PV(j) follows
-        // once both heads' P(j) are written.  Queue: ... PV(j-1), QK(j+1), PV(j) ...
-        for (int j = 0; ok && j < n_kt; ++j) {
-          const int s = j % C::kStages;
-          if (j + 1 < n_kt) {
-            const int s1 = (j + 1) % C::kStages;
-            ok = wait(bars.s_free, j & 1, 5) && wait(bars.k_full + s1, ((j + 1) / C::kStages) & 1, 6);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t kl = k_lo + s1 * kKVStep, kxl = kx_lo + s1 * kXStep;
-            if (nh == 2) issue_qk<D, 2>(tmem, 0, q_lo, kl, qx_lo, kxl, idesc_qk);
-            else issue_qk<D, 1>(tmem, 0, q_lo, kl, qx_lo, kxl, idesc_qk);
-            umma_commit(bars.s_full);
-            umma_commit(bars.k_empty + s1);
-          }
-          ok = wait(bars.p_ready, j & 1, 7) && wait(bars.v_full + s, (j / C::kStages) & 1, 8);
+          // Both heads in lockstep (one S/P/O barrier set for the pair).  The
+          // softmax releases S right after reading it, so QK(j+1) goes in as
+          // soon as that happens and runs during the softmax of tile j; PV(j)
+          // follows once both heads' P(j) are written.  Queue: ... PV(j-1),
+          // QK(j+1), PV(j) ...; the next item's first QK follows the current
+          // item's last PV, and runs while the softmax warps write the output.
+          ok = (g == 0 || wait(bars.s_free, (g - 1) & 1, 5)) &&
+               wait(bars.k_full + g % C::kStages, (g / C::kStages) & 1, 1);
           if (!ok) break;
           tc_fence_after();
-          if (nh == 2) issue_pv<D, 2, true>(tmem, 0, v_lo + s * kKVStep, idesc_pv, j == 0);
-          else issue_pv<D, 1, true>(tmem, 0, v_lo + s * kKVStep, idesc_pv, j == 0);
-          umma_commit(bars.o_done);
-          umma_commit(bars.v_empty + s);
-        }
-      } else {
-        // P is written over S, so QK_h(j+1) can only follow PV_h(j).  Fixed
-        // ping-pong order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1): while one
-        // head's softmax runs, the tensor core works through the other head's
-        // PV and next QK.
-        for (int j = 0; ok && j < n_kt; ++j) {
-          const int s = j % C::kStages, s1 = (j + 1) % C::kStages;
-          for (int h = 0; ok && h < nh; ++h) {
-            ok = wait(bars.p_ready + h, j & 1, 7) && (h > 0 || wait(bars.v_full + s, (j / C::kStages) & 1, 8));
-            if (!ok) break;
-            tc_fence_after();
-            issue_pv<D, 1, false>(tmem, h, v_lo + s * kKVStep, idesc_pv, j == 0);
-            umma_commit(bars.o_done + h);
+          {
+            const uint32_t kl = k_lo + (g % C::kStages) * kKVStep, kxl = kx_lo + (g % C::kStages) * kXStep;
+            if (nh == 2) issue_qk<D, 2>(tmem, 0, q_lo, kl, qx_lo, kxl, idesc_qk);
+            else issue_qk<D, 1>(tmem, 0, q_lo, kl, qx_lo, kxl, idesc_qk);
+          }
+          umma_commit(bars.s_full);
+          umma_commit(bars.k_empty + g % C::kStages);
+          if (n_kt == 1) umma_commit(bars.q_empty);
+          for (int j = 0; ok && j < n_kt; ++j) {
+            const int gt = g + j, s = gt % C::kStages;
             if (j + 1 < n_kt) {
-              ok = h > 0 || wait(bars.k_full + s1, ((j + 1) / C::kStages) & 1, 6);
+              const int s1 = (gt + 1) % C::kStages;
+              ok = wait(bars.s_free, gt & 1, 5) && wait(bars.k_full + s1, ((gt + 1) / C::kStages) & 1, 6);
               if (!ok) break;
               tc_fence_after();
-              issue_qk<D, 1>(tmem, h, q_lo, k_lo + s1 * kKVStep, qx_lo, kx_lo + s1 * kXStep, idesc_qk);
-              umma_commit(bars.s_full + h);
+              const uint32_t kl = k_lo + s1 * kKVStep, kxl = kx_lo + s1 * kXStep;
+              if (nh == 2) issue_qk<D, 2>(tmem, 0, q_lo, kl, qx_lo, kxl, idesc_qk);
+              else issue_qk<D, 1>(tmem, 0, q_lo, kl, qx_lo, kxl, idesc_qk);
+              umma_commit(bars.s_full);
+              umma_commit(bars.k_empty + s1);
+              if (j + 2 == n_kt) umma_commit(bars.q_empty);
+            }
+            ok = wait(bars.p_ready, gt & 1, 7) && wait(bars.v_full + s, (gt / C::kStages) & 1, 8);
+            if (!ok) break;
+            tc_fence_after();
+            if (nh == 2) issue_pv<D, 2, true>(tmem, 0, v_lo + s * kKVStep, idesc_pv, j == 0);
+            else issue_pv<D, 1, true>(tmem, 0, v_lo + s * kKVStep, idesc_pv, j == 0);
+            umma_commit(bars.o_done);
+            umma_commit(bars.v_empty + s);
+          }
+        } else {
+          // P is written over S, so QK_h(j+1) can only follow PV_h(j).  Fixed
+          // ping-pong order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1): while one
+          // head's softmax runs, the tensor core works through the other head's
+          // PV and next QK.  Head 0 counts every key tile, head 1 only those of
+          // items where the pair has two heads.
+          ok = wait(bars.k_full + g % C::kStages, (g / C::kStages) & 1, 1);
+          if (!ok) break;
+          tc_fence_after();
+          for (int h = 0; h < nh; ++h) {
+            issue_qk<D, 1>(tmem, h, q_lo, k_lo + (g % C::kStages) * kKVStep, qx_lo,
+                           kx_lo + (g % C::kStages) * kXStep, idesc_qk);
+            umma_commit(bars.s_full + h);
+          }
+          umma_commit(bars.k_empty + g % C::kStages);
+          if (n_kt == 1) umma_commit(bars.q_empty);
+          for (int j = 0; ok && j < n_kt; ++j) {
+            const int gt = g + j, s = gt % C::kStages, s1 = (gt + 1) % C::kStages;
+            for (int h = 0; ok && h < nh; ++h) {
+              const int ph = h == 0 ? gt : t1 + j;
+              ok = wait(bars.p_ready + h, ph & 1, 7) && (h > 0 || wait(bars.v_full + s, (gt / C::kStages) & 1, 8));
+              if (!ok) break;
+              tc_fence_after();
+              issue_pv<D, 1, false>(tmem, h, v_lo + s * kKVStep, idesc_pv, j == 0);
+              umma_commit(bars.o_done + h);
+              if (j + 1 < n_kt) {
+                ok = h > 0 || wait(bars.k_full + s1, ((gt + 1) / C::kStages) & 1, 6);
+                if (!ok) break;
+                tc_fence_after();
+                issue_qk<D, 1>(tmem, h, q_lo, k_lo + s1 * kKVStep, qx_lo, kx_lo + s1 * kXStep, idesc_qk);
+                umma_commit(bars.s_full + h);
+              }
+            }
+            if (!ok) break;
+            umma_commit(bars.v_empty + s);
+            if (j + 1 < n_kt) {
+              umma_commit(bars.k_empty + s1);
+              if (j + 2 == n_kt) umma_commit(bars.q_empty);
             }
           }
-          if (!ok) break;
-          umma_commit(bars.v_empty + s);
-          if (j + 1 < n_kt) umma_commit(bars.k_empty + s1);
+          if (nh == 2) t1 += n_kt;
         }
+        g += n_kt;
       }
       if (!ok) *abort_flag = 1;
       // drain every MMA before TMEM is released
@@ -517,20 +605,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
     const uint32_t tS = tmem + lane_base + h * 128;
     const uint32_t tO = tmem + lane_base + 256 + h * D;
-    const bool row_valid = row < nrows;
-    if (h < nh) {
+    // barrier index: the lockstep layout (separate P) has one set for the pair
+    const int hb = C::kSepP ? 0 : h;
+    const unsigned long long scale2 = f32x2(scale_log2, scale_log2);
+    bool ok = true;
+    int g = 0, th = 0;   // key tiles so far (all items), key tiles this head took part in
+    ItemInfo x;
+    for (int i = 0; ok && item_info(i, x); ++i) {
+      const int n_kt = x.n_kt;
+      if (n_kt == 0) continue;
+      if (h >= x.nh) {
+        if (C::kSepP && hw == 2) {
+          // the pair has one head: keep the lockstep barriers' counts
+          for (int j = 0; ok && j < n_kt; ++j) {
+            const int gt = g + j;
+            ok = mbar_wait(bars.s_full, gt & 1, err, kDevErrTimeoutBase + 10) && !aborted(abort_flag);
+            if (!ok) break;
+            mbar_arrive(bars.s_free);
+            mbar_arrive(bars.p_ready);
+            // the next tile's arrivals must not reach this tile's phases
+            ok = mbar_wait(bars.o_done, gt & 1, err, kDevErrTimeoutBase + 11);
+          }
+          if (!ok) *abort_flag = 1;
+        }
+        g += n_kt;
+        continue;
+      }
+      const int ph0 = C::kSepP ? g : th;   // phase counter of this head's S/P/O barriers
+      const int n_full = x.n_full;
+      const int r0 = x.it.t * kRowTile;
+      const int nrows = min(kRowTile, L - r0);
+      const bool row_valid = row < nrows;
       float m = -INFINITY, l = 0.0f;
-      bool ok = true;
-      const unsigned long long scale2 = f32x2(scale_log2, scale_log2);
-      // barrier index: the lockstep layout (separate P) has one set for the pair
-      const int hb = C::kSepP ? 0 : h;
       for (int j = 0; j < n_kt; ++j) {
-        const int ms_slot = j % C::kMetaSlots;
-        ok = mbar_wait(bars.s_full + hb, j & 1, err, kDevErrTimeoutBase + 10);
+        const int gt = g + j, ph = ph0 + j;
+        const int ms_slot = gt % C::kMetaSlots;
+        ok = mbar_wait(bars.s_full + hb, ph & 1, err, kDevErrTimeoutBase + 10);
         // the tile's row-interval table (published by the K producer)
-        if (ok) ok = mbar_wait(bars.meta_full + ms_slot, (j / C::kMetaSlots) & 1, err, kDevErrTimeoutBase + 13);
+        if (ok) ok = mbar_wait(bars.meta_full + ms_slot, (gt / C::kMetaSlots) & 1, err, kDevErrTimeoutBase + 13);
         if (!ok || aborted(abort_flag)) {
-          *abort_flag = 1;
+          ok = false;
           break;
         }
         tc_fence_after();
@@ -601,11 +715,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 64; ++c) pk[c] = p_pair(2 * c);
           if (j > 0) {
-            ok = mbar_wait(bars.o_done, (j - 1) & 1, err, kDevErrTimeoutBase + 11);
-            if (!ok) {
-              *abort_flag = 1;
-              break;
-            }
+            ok = mbar_wait(bars.o_done, (gt - 1) & 1, err, kDevErrTimeoutBase + 11);
+            if (!ok) break;
             tc_fence_after();
           }
           const uint32_t tP = tmem + lane_base + 384 + h * 64;
@@ -623,9 +734,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           // consume every o_done phase in order (PV of the previous tile), so
           // the parity of the epilogue's wait is never ambiguous
           if (j > 0) {
-            ok = mbar_wait(bars.o_done + h, (j - 1) & 1, err, kDevErrTimeoutBase + 11);
+            ok = mbar_wait(bars.o_done + h, (ph - 1) & 1, err, kDevErrTimeoutBase + 11);
             if (!ok) {
-              *abort_flag = 1;
               tmem_wait_st();
               break;
             }
@@ -655,34 +765,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(bars.p_ready + hb);
       }
-      // epilogue
-      if (ok && !aborted(abort_flag) && n_kt > 0) {
-        ok = mbar_wait(bars.o_done + hb, (n_kt - 1) & 1, err, kDevErrTimeoutBase + 12);
-        if (ok) {
-          tc_fence_after();
-          const float inv = 1.0f / l;
-          uint16_t* orow = out + ((static_cast<size_t>(b) * L + r0 + row) * Hq + h0 + h) * D;
+      // epilogue: O / l once PV of the item's last key tile is done
+      if (ok) ok = mbar_wait(bars.o_done + hb, (ph0 + n_kt - 1) & 1, err, kDevErrTimeoutBase + 12);
+      if (!ok) break;
+      tc_fence_after();
+      const float inv = 1.0f / l;
+      uint16_t* orow =
+          out + ((static_cast<size_t>(x.it.b) * L + r0 + row) * Hq + x.it.g * nrep + 2 * x.it.pair + h) * D;
 #pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o[32];
-            DMA_TMEM_LD32(tO + c0, o);
-            tmem_wait_ld();
-            if (row_valid) {
-              uint32_t pk2[16];
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        DMA_TMEM_LD32(tO + c0, o);
+        tmem_wait_ld();
+        if (row_valid) {
+          uint32_t pk2[16];
 #pragma unroll
-              for (int c = 0; c < 16; ++c)
-                pk2[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv, __uint_as_float(o[2 * c + 1]) * inv);
+          for (int c = 0; c < 16; ++c)
+            pk2[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv, __uint_as_float(o[2 * c + 1]) * inv);
 #pragma unroll
-              for (int c = 0; c < 4; ++c)
-                *reinterpret_cast<uint4*>(orow + c0 + c * 8) =
-                    make_uint4(pk2[4 * c], pk2[4 * c + 1], pk2[4 * c + 2], pk2[4 * c + 3]);
-            }
-          }
-        } else {
-          *abort_flag = 1;
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(orow + c0 + c * 8) =
+                make_uint4(pk2[4 * c], pk2[4 * c + 1], pk2[4 * c + 2], pk2[4 * c + 3]);
         }
       }
+      // O may be overwritten by the next item's first PV (after this thread's
+      // next p_ready arrival)
+      tc_fence_before();
+      g += n_kt;
+      th += n_kt;
     }
+    if (!ok) *abort_flag = 1;
   }
 
   tc_fence_before();
@@ -758,7 +870,13 @@ cudaError_t launch_d(const void* q, const void* k, const void* v, const Geometry
   if (e != cudaSuccess) return e;
   const int nrep = g.Hq / g.Hkv;
   const int npairs = (nrep + 1) / 2;
-  const long long nblocks = static_cast<long long>(plan.n_row_tiles) * g.B * g.Hkv * npairs;
+  const long long n_items = static_cast<long long>(plan.n_row_tiles) * g.B * g.Hkv * npairs;
+  if (n_items > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  int dev = 0, nsm = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return cudaErrorInvalidDevice;
+  const long long nblocks = n_items < nsm ? n_items : nsm;   // persistent: one CTA per SM
   attn_prefill_kernel<D><<<static_cast<unsigned>(nblocks), kThreads, C::kSmemBytes, s>>>(
       tq, tk, tv, tk3, tv3, plan, g.B, g.Lk, g.Hq, g.Hkv, scale * kLog2e, 1.0f / scale, static_cast<uint16_t*>(out),
       err);

@@ -46,9 +46,18 @@
 namespace dma {
 namespace {
 
-constexpr int kThreads = 352;   // 11 warps: K producer, MMA/TMEM, V producer, 2 x 4 softmax
-// (registers come from each SM sub-partition's own file: with 11 warps three share one, so
-// 168 per thread is the most one CTA per SM can have)
+// 12 warps in three warpgroups: warpgroup 0 = K producer, MMA issuer (and TMEM
+// owner), V producer and one spare warp; warpgroups 1 and 2 = the softmax of the
+// pair's two heads (four warps each, one per TMEM lane quarter).  The block is
+// launched with at most 168 registers per thread; warpgroup 0 then gives
+// registers back (setmaxnreg.dec) and the softmax warpgroups take them
+// (setmaxnreg.inc), so the 128-column score row and its probabilities stay in
+// registers.  128 x kRegsControl + 256 x kRegsSoftmax must not exceed what the
+// block was launched with: the launcher checks it before every launch.
+constexpr int kThreads = 384;
+constexpr int kRegsControl = 72;
+constexpr int kRegsSoftmax = 208;
+static_assert(kRegsControl % 8 == 0 && kRegsSoftmax % 8 == 0, "setmaxnreg takes multiples of 8");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 // every kPolyEvery-th pair of probabilities in a row is computed on the FMA pipe
@@ -300,10 +309,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmap_k3);
     prefetch_tmap(&tmap_v3);
   }
-  if (warp >= 3) {
+  if (warp >= 4) {
     // constant parts of the extra K=16 block: Q's columns of ones, the zero
     // half of every key stage's bias block
-    const int i = threadIdx.x - 96;    // 0..255
+    const int i = threadIdx.x - 128;    // 0..255
     const int r = i & 127;
     const int hq = i >> 7;
     *reinterpret_cast<uint4*>(sQx + hq * kXBytes + xoff(r, 0)) = make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u);
@@ -336,6 +345,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     return true;
   };
 
+  if (warp < 4) {
+  // warpgroup 0 gives registers back to the softmax warpgroups
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
   if (warp == 0) {
     // ======================= K producer =====================================
     int gk = 0, nq = 0;   // K tiles and Q tiles issued so far
@@ -598,9 +610,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_hot(bars.fin, 0, err, kDevErrTimeoutBase + 9);
     }
     __syncwarp();
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // ======================= softmax / epilogue ============================
-    const int h = (warp - 3) / 4;             // which head of the pair (warps 3-6, 7-10)
+    const int h = (warp - 4) / 4;             // which head of the pair (warps 4-7, 8-11)
     const int row = (warp % 4) * 32 + lane;   // TMEM lane = query row in the tile
     const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
     const uint32_t tS = tmem + lane_base + h * 128;
@@ -616,15 +630,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (n_kt == 0) continue;
       if (h >= x.nh) {
         if (C::kSepP && hw == 2) {
-          // the pair has one head: keep the lockstep barriers' counts
+          // the pair has one head: keep the lockstep barriers' counts, in the
+          // same order as a working head (s_free as soon as S is there; p_ready
+          // only after PV of the previous tile, so it cannot count toward that
+          // tile's phase)
           for (int j = 0; ok && j < n_kt; ++j) {
             const int gt = g + j;
             ok = mbar_wait(bars.s_full, gt & 1, err, kDevErrTimeoutBase + 10) && !aborted(abort_flag);
             if (!ok) break;
             mbar_arrive(bars.s_free);
+            if (j > 0) ok = mbar_wait(bars.o_done, (gt - 1) & 1, err, kDevErrTimeoutBase + 11);
+            if (!ok) break;
             mbar_arrive(bars.p_ready);
-            // the next tile's arrivals must not reach this tile's phases
-            ok = mbar_wait(bars.o_done, gt & 1, err, kDevErrTimeoutBase + 11);
           }
           if (!ok) *abort_flag = 1;
         }
@@ -868,6 +885,13 @@ cudaError_t launch_d(const void* q, const void* k, const void* v, const Geometry
   cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;
+  {
+    // the warpgroups' register split must fit in what the block is launched with
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, attn_prefill_kernel<D>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * kThreads < 128 * kRegsControl + 256 * kRegsSoftmax) return cudaErrorInvalidConfiguration;
+  }
   const int nrep = g.Hq / g.Hkv;
   const int npairs = (nrep + 1) / 2;
   const long long n_items = static_cast<long long>(plan.n_row_tiles) * g.B * g.Hkv * npairs;

@@ -52,7 +52,7 @@ __device__ __forceinline__ int clamp_len(const int32_t* lengths, int b, int L, u
   return len;
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_prefill_kernel(const float* __restrict__ dt,
+__global__ void __launch_bounds__(kSelThreads, 2) select_prefill_kernel(const float* __restrict__ dt,
                                                                      const int32_t* __restrict__ lengths, int Hkv,
                                                                      int L, int w, PrefillPlan plan,
                                                                      uint32_t* err) {
@@ -106,9 +106,9 @@ __global__ void __launch_bounds__(kSelThreads) select_prefill_kernel(const float
   const int n_old = p + 1 > w ? w : p + 1;
 
   // 2. the union U of kept keys, in index order
-  const int nU = ordered_compact(
-      q + 1, [&](int j) { return composite_key(bits[j], j) >= tau0; },
-      [&](int pos, int j) { U[pos] = composite_key(bits[j], j); }, sc);
+  const int nU = ordered_compact_row(
+      bits, q + 1, [&](uint32_t v, int j) { return composite_key(v, j) >= tau0; },
+      [&](int pos, int j, uint32_t v) { U[pos] = composite_key(v, j); }, sc);
   __syncthreads();
 
   // 3. the kRowTile smallest keys of U, ascending; then tau for every row
@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(kSelThreads) select_prefill_kernel(const float
   }
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_decode_kernel(const float* __restrict__ dt,
+__global__ void __launch_bounds__(kSelThreads, 4) select_decode_kernel(const float* __restrict__ dt,
                                                                     const int32_t* __restrict__ lengths, int Hkv,
                                                                     int Lk, int w, DecodePlan plan, uint32_t* err) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -240,11 +240,11 @@ __global__ void __launch_bounds__(kSelThreads) select_decode_kernel(const float*
   uint64_t tau = 0ull;
   if (Lk > w && len > w) {
     tau = select_kth_global(bits, len, static_cast<uint32_t>(w), sc);
-    n = ordered_compact(
-        len, [&](int j) { return composite_key(bits[j], j) >= tau; },
-        [&](int pos, int j) {
+    n = ordered_compact_row(
+        bits, len, [&](uint32_t v, int j) { return composite_key(v, j) >= tau; },
+        [&](int pos, int j, uint32_t v) {
           idx_o[pos] = j;
-          bias_o[pos] = __uint_as_float(bits[j]);
+          bias_o[pos] = __uint_as_float(v);
         },
         sc);
   } else {

@@ -184,15 +184,55 @@ __device__ __noinline__ int kth_matching_index(const uint32_t* __restrict__ bits
   return r;
 }
 
+// Visits every position j in [0, n) of a dt row as f(bits, j, valid), each
+// thread a strided subset.  A 16-byte-aligned row is read four keys per 16-byte
+// load, four loads in flight per thread, so a pass over a long row is limited by
+// bandwidth rather than by one load's latency per key.  Every thread of the
+// block makes the same number of calls (valid = false past the end), so f may
+// use warp-wide votes.
+template <class F>
+__device__ __forceinline__ void row_for_each(const uint32_t* __restrict__ bits, int n, F&& f) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  int done = 0;
+  if ((reinterpret_cast<uintptr_t>(bits) & 15u) == 0) {
+    const int nq = n >> 2;
+    const uint4* q = reinterpret_cast<const uint4*>(bits);
+    for (int r0 = 0; r0 < nq; r0 += 4 * nt) {   // same trip count in every thread
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = r0 + u * nt + tid;
+        v[u] = i < nq ? __ldg(q + i) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = r0 + u * nt + tid;
+        const bool ok = i < nq;
+        f(v[u].x, 4 * i, ok);
+        f(v[u].y, 4 * i + 1, ok);
+        f(v[u].z, 4 * i + 2, ok);
+        f(v[u].w, 4 * i + 3, ok);
+      }
+    }
+    done = nq << 2;
+  }
+  for (int j0 = done; j0 < n; j0 += nt) {
+    const int j = j0 + tid;
+    const bool ok = j < n;
+    f(ok ? __ldg(bits + j) : 0u, j, ok);
+  }
+}
+
 // k-th largest composite key (1 <= k <= n) among positions [0, n) of a dt row.
 __device__ __noinline__ uint64_t select_kth_global(const uint32_t* __restrict__ bits, int n, uint32_t k,
                                                    SelScratch sc) {
-  uint64_t vor = 0, vand = ~0ull;
-  for (int j = threadIdx.x; j < n; j += blockDim.x) {
-    const uint64_t b = bits[j];
-    vor |= b;
-    vand &= b;
-  }
+  uint32_t vor = 0u, vand = ~0u;
+  row_for_each(bits, n, [&](uint32_t b, int, bool ok) {
+    if (ok) {
+      vor |= b;
+      vand &= b;
+    }
+  });
   uint64_t O, A;
   block_or_and64(vor, vand, sc.red, O, A);
   O &= 0xFFFFFFFFull;
@@ -206,10 +246,9 @@ __device__ __noinline__ uint64_t select_kth_global(const uint32_t* __restrict__ 
     const int nb = 1 << (hb - s + 1);
     for (int i = threadIdx.x; i < nb; i += blockDim.x) sc.hist[i] = 0;
     __syncthreads();
-    for (int j = threadIdx.x; j < n; j += blockDim.x) {
-      const uint64_t b = bits[j];
-      if (hi_match(b, prefix, hb)) atomicAdd(&sc.hist[(b >> s) & static_cast<uint64_t>(nb - 1)], 1u);
-    }
+    row_for_each(bits, n, [&](uint32_t b, int, bool ok) {
+      if (ok && hi_match(b, prefix, hb)) atomicAdd(&sc.hist[(b >> s) & static_cast<uint32_t>(nb - 1)], 1u);
+    });
     __syncthreads();
     uint32_t kk, cnt;
     const uint32_t B = find_bin_from_top(sc.hist, nb, k, sc.red, sc.vars, &kk, &cnt);
@@ -221,13 +260,22 @@ __device__ __noinline__ uint64_t select_kth_global(const uint32_t* __restrict__ 
   if (count <= static_cast<uint32_t>(kCandCap)) {
     if (threadIdx.x == 0) sc.vars[7] = 0;
     __syncthreads();
-    for (int j = threadIdx.x; j < n; j += blockDim.x) {
-      const uint64_t b = bits[j];
-      if (hi_match(b, prefix, hb)) {
-        const uint32_t pos = atomicAdd(reinterpret_cast<unsigned long long*>(&sc.vars[7]), 1ull);
-        if (pos < static_cast<uint32_t>(kCandCap)) sc.cand[pos] = composite_key(static_cast<uint32_t>(b), j);
+    // candidates appended with one shared-memory atomic per warp and vote
+    const uint32_t lane = lane_id();
+    row_for_each(bits, n, [&](uint32_t b, int j, bool ok) {
+      const bool m = ok && hi_match(b, prefix, hb);
+      const uint32_t vote = __ballot_sync(0xFFFFFFFFu, m);
+      if (vote) {
+        uint32_t base = 0;
+        if (lane == 0) base = static_cast<uint32_t>(
+            atomicAdd(reinterpret_cast<unsigned long long*>(&sc.vars[7]), static_cast<unsigned long long>(__popc(vote))));
+        base = __shfl_sync(0xFFFFFFFFu, base, 0);
+        if (m) {
+          const uint32_t pos = base + __popc(vote & lanemask_lt());
+          if (pos < static_cast<uint32_t>(kCandCap)) sc.cand[pos] = composite_key(b, j);
+        }
       }
-    }
+    });
     __syncthreads();
     const int c = static_cast<int>(sc.vars[7]);
     __syncthreads();
@@ -270,6 +318,83 @@ __device__ __forceinline__ int ordered_compact(int n, Pred pred, Emit emit, SelS
     const uint32_t m = __ballot_sync(0xFFFFFFFFu, p);
     if (p) emit(static_cast<int>(run + __popc(m & lanemask_lt())), j);
     run += __popc(m);
+  }
+  const int total = static_cast<int>(sc.red[32]);
+  __syncthreads();
+  return total;
+}
+
+// Stable compaction over a dt row: emit(pos, j, bits[j]) for the positions j
+// in [0, n) with pred(bits[j], j), pos = 0, 1, ... in increasing j; returns
+// the count.  Each warp owns a contiguous segment, read as 16-byte quads (a
+// lane holds four consecutive keys), with two quads in flight per lane.
+template <class Pred, class Emit>
+__device__ __forceinline__ int ordered_compact_row(const uint32_t* __restrict__ bits, int n, Pred pred, Emit emit,
+                                                   SelScratch sc) {
+  if ((reinterpret_cast<uintptr_t>(bits) & 15u) != 0)
+    return ordered_compact(
+        n, [&](int j) { return pred(bits[j], j); }, [&](int pos, int j) { emit(pos, j, bits[j]); }, sc);
+  const uint32_t lane = lane_id(), warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int seg = ((n + nw - 1) / nw + 127) / 128 * 128;
+  const int s0 = warp * seg, s1 = min(n, s0 + seg);
+  // the four keys of this lane at chunk start c0 (positions past s1 read as 0)
+  auto load4 = [&](int c0, uint32_t (&v)[4]) {
+    const int j = c0 + 4 * static_cast<int>(lane);
+    if (j + 3 < s1) {
+      const uint4 q = __ldg(reinterpret_cast<const uint4*>(bits + j));
+      v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] = j + e < s1 ? __ldg(bits + j + e) : 0u;
+    }
+  };
+  uint32_t cnt = 0;
+  for (int c0 = s0; c0 < s1; c0 += 256) {
+    uint32_t v0[4], v1[4];
+    load4(c0, v0);
+    load4(c0 + 128, v1);
+    const int j = c0 + 4 * static_cast<int>(lane);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      cnt += (j + e < s1 && pred(v0[e], j + e)) ? 1u : 0u;
+      cnt += (j + 128 + e < s1 && pred(v1[e], j + 128 + e)) ? 1u : 0u;
+    }
+  }
+  cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
+  __syncthreads();
+  if (lane == 0) sc.red[warp] = cnt;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t acc = 0;
+    for (uint32_t w = 0; w < nw; ++w) {
+      const uint32_t c = sc.red[w];
+      sc.red[w] = acc;
+      acc += c;
+    }
+    sc.red[32] = acc;
+  }
+  __syncthreads();
+  uint32_t run = sc.red[warp];
+  const uint32_t lt = lanemask_lt();
+  for (int c0 = s0; c0 < s1; c0 += 128) {
+    uint32_t v[4];
+    load4(c0, v);
+    const int j = c0 + 4 * static_cast<int>(lane);
+    bool p[4];
+    uint32_t c = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      p[e] = j + e < s1 && pred(v[e], j + e);
+      c += p[e] ? 1u : 0u;
+    }
+    // exclusive prefix of c (0..4) over the lanes, from its three bits
+    const uint32_t b0 = __ballot_sync(0xFFFFFFFFu, c & 1u), b1 = __ballot_sync(0xFFFFFFFFu, c & 2u),
+                   b2 = __ballot_sync(0xFFFFFFFFu, c & 4u);
+    uint32_t pos = run + __popc(b0 & lt) + 2u * __popc(b1 & lt) + 4u * __popc(b2 & lt);
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (p[e]) emit(static_cast<int>(pos++), j + e, v[e]);
+    run += __popc(b0) + 2u * __popc(b1) + 4u * __popc(b2);
   }
   const int total = static_cast<int>(sc.red[32]);
   __syncthreads();

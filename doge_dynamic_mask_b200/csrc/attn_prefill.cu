@@ -822,24 +822,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---- host: tensor maps -------------------------------------------------------
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
 template <int D>
 cudaError_t launch_d(const void* q, const void* k, const void* v, const Geometry& g, float scale,
                      const PrefillPlan& plan, void* out, uint32_t* err, cudaStream_t s) {
@@ -908,6 +890,20 @@ cudaError_t launch_d(const void* q, const void* k, const void* v, const Geometry
 }
 
 }  // namespace
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
 
 cudaError_t launch_attn_prefill(const void* q, const void* k, const void* v, const Geometry& g, float scale,
                                 const PrefillPlan& plan, void* out, uint32_t* err, cudaStream_t s) {

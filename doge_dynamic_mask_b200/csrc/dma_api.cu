@@ -175,7 +175,7 @@ dma_status_t dma_dt_scores(const void* v, const float* W_dt, const float* A, int
   dma_status_t st = check_shape(B, L, Hkv, Hkv, d, 1);
   if (st != DMA_OK) return st;
   if ((st = device_ok()) != DMA_OK) return st;
-  cudaError_t e = launch_dt_scores(v, W_dt, A, B, L, Hkv, d, dt_out, reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_dt_scores(v, W_dt, A, B, L, Hkv, d, dt_out, nullptr, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DMA_OK : cuda_fail(e);
 }
 
@@ -249,7 +249,7 @@ dma_status_t dma_forward_prefill(const void* q, const void* k, const void* v, co
   const float* dt = dt_in;
   if ((e = stage_mark(0, s)) != cudaSuccess) return cuda_fail(e);
   if (!dt) {
-    if ((e = launch_dt_scores(v, W_dt, A, B, L, Hkv, d, plan.dt, s)) != cudaSuccess) return cuda_fail(e);
+    if ((e = launch_dt_scores(v, W_dt, A, B, L, Hkv, d, plan.dt, err, s)) != cudaSuccess) return cuda_fail(e);
     dt = plan.dt;
   }
   if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e);
@@ -283,7 +283,7 @@ dma_status_t dma_decode_step(const void* q, const void* k_cache, const void* v_c
   const float* dt = dt_in;
   if ((e = stage_mark(0, s)) != cudaSuccess) return cuda_fail(e);
   if (!dt) {
-    if ((e = launch_dt_scores(v_cache, W_dt, A, B, Lk, Hkv, d, plan.dt, s)) != cudaSuccess) return cuda_fail(e);
+    if ((e = launch_dt_scores(v_cache, W_dt, A, B, Lk, Hkv, d, plan.dt, err, s)) != cudaSuccess) return cuda_fail(e);
     dt = plan.dt;
   }
   if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e);

@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace dma {
@@ -76,9 +77,16 @@ size_t decode_plan_bytes(const Geometry& g);
 PrefillPlan carve_prefill_plan(void* ws, const Geometry& g);
 DecodePlan carve_decode_plan(void* ws, const Geometry& g);
 
-// launchers (return cudaGetLastError() after the launch)
+// cuTensorMapEncodeTiled from the driver (through the runtime's entry-point
+// query, so the library links no driver stub); nullptr when unavailable.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_fn();
+
+// launchers (return cudaGetLastError() after the launch); err: device status word or nullptr
 cudaError_t launch_dt_scores(const void* v, const float* W, const float* A, int B, int L, int Hkv, int d,
-                             float* dt, cudaStream_t s);
+                             float* dt, uint32_t* err, cudaStream_t s);
 cudaError_t launch_select_prefill(const float* dt, const int32_t* lengths, const Geometry& g,
                                   const PrefillPlan& plan, uint32_t* err, cudaStream_t s);
 cudaError_t launch_select_decode(const float* dt, const int32_t* lengths, const Geometry& g,

@@ -18,6 +18,18 @@
 // the matching pair of value channels.  The epilogue adds the two halves,
 // applies softplus, the A multiply and exp in float32 and writes dt
 // [B, Hkv, L] coalesced across lanes.
+//
+// Tensor-core path (Hkv <= 8, d in {64, 128}).  The same projection as a
+// [tokens x C] x [C x N] product on tcgen05 tensor cores, so the kernel is
+// bound by streaming V from HBM rather than by float32 FMA issue: a persistent
+// CTA per SM streams 128-token tiles of V through an 8-stage ring of 16 KB
+// shared-memory stages (TMA, 128-byte swizzle, 64 channels per stage); one
+// thread issues M=128, K=16 MMAs into a double-buffered TMEM accumulator; four
+// epilogue warps finish the tiles.  B holds the float32 weight split exactly
+// into three bf16 terms, W = W_hi + W_mid + W_lo (each the bf16 rounding of
+// what the previous terms leave), as column groups [W_hi | W_mid | W_lo]:
+// products of bf16 values are exact and the tensor core accumulates in
+// float32, so the three column sums add up to the float32 projection.
 #include "common.cuh"
 
 namespace dma {
@@ -45,10 +57,6 @@ __device__ __forceinline__ unsigned long long bf16x2_to_f32x2(uint32_t u) {
 __device__ __forceinline__ float softplus_f32(float x) {
   // log(1 + e^x) in the overflow-free form max(x, 0) + log1p(e^-|x|).
   return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
-}
-
-__device__ __forceinline__ uint32_t word(const uint4& u, int i) {
-  return i == 0 ? u.x : i == 1 ? u.y : i == 2 ? u.z : u.w;
 }
 
 // 32 bytes (16 bf16 channels) of one token row.  WIDE: one 256-bit load (the
@@ -191,10 +199,245 @@ cudaError_t launch_t(const void* v, const float* W, const float* A, int B, int L
               : launch_k<HKV, D, KBIG, false>(v, W, A, ntok, L, dt, nsm, s);
 }
 
+
+// ---- tensor-core path ---------------------------------------------------------
+
+__device__ __forceinline__ bool aborted_flag(volatile int* flag) { return *flag != 0; }
+
+constexpr int kDtTcThreads = 192;   // warp 0: TMA producer; warp 1: MMA issuer, TMEM owner; warps 2-5: epilogue
+constexpr int kDtTile = 128;        // tokens per tile (MMA M)
+constexpr int kDtStages = 8;
+constexpr int kDtChunk = 64;        // channels per stage: one 128-byte swizzled row per token
+
+template <int HKV, int D>
+struct DtTc {
+  static constexpr int C = HKV * D;
+  static constexpr int kChunks = C / kDtChunk;
+  static constexpr int N = (3 * HKV + 15) / 16 * 16;     // three bf16 terms per head, padded for the MMA
+  static constexpr int kStageBytes = kDtTile * 128;      // 16 KB
+  static constexpr int kBChunkBytes = N * 128;           // B rows (N) x 64 channels
+  static constexpr int kOffA = kChunks * kBChunkBytes;
+  static constexpr int kOffBar = kOffA + kDtStages * kStageBytes;
+  static constexpr int kSmemBytes = kOffBar + 256 + 1024;   // + alignment slack
+  static constexpr uint32_t kTmemCols = 2 * N <= 32 ? 32 : (2 * N <= 64 ? 64 : 128);
+  static_assert(kBChunkBytes % 1024 == 0, "swizzle atoms need 1024-byte aligned chunks");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+// byte offset of element (row n, channel c) of B in the K-major 128-byte-swizzled layout
+template <int N>
+__device__ __forceinline__ uint32_t b_offset(int n, int c) {
+  const int kc = c / kDtChunk, cc = c % kDtChunk;
+  return static_cast<uint32_t>(kc * N * 128 + n * 128 + (((cc >> 3) ^ (n & 7)) << 4) + (cc & 7) * 2);
+}
+
+template <int HKV, int D>
+__global__ void __launch_bounds__(kDtTcThreads, 1)
+    dt_tc_kernel(const __grid_constant__ CUtensorMap tmap_v, const float* __restrict__ W,
+                 const float* __restrict__ A, int ntok, int L, float* __restrict__ dt, uint32_t* err) {
+  using T = DtTc<HKV, D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                         ~static_cast<uintptr_t>(1023));
+  unsigned char* sB = smem;
+  unsigned char* sA = smem + T::kOffA;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + T::kOffBar);
+  uint64_t* empty = full + kDtStages;
+  uint64_t* acc_full = empty + kDtStages;    // [2]
+  uint64_t* acc_empty = acc_full + 2;        // [2]
+  uint64_t* fin = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = (ntok + kDtTile - 1) / kDtTile;
+
+  // B = [W_hi | W_mid | W_lo | 0], row n = term * HKV + g, K-major over the channels
+  for (int i = threadIdx.x; i < T::C * HKV; i += blockDim.x) {
+    const int c = i / HKV, g = i % HKV;
+    const float w = W[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+    *reinterpret_cast<__nv_bfloat16*>(sB + b_offset<T::N>(g, c)) = hi;
+    *reinterpret_cast<__nv_bfloat16*>(sB + b_offset<T::N>(HKV + g, c)) = mid;
+    *reinterpret_cast<__nv_bfloat16*>(sB + b_offset<T::N>(2 * HKV + g, c)) = lo;
+  }
+  for (int i = threadIdx.x; i < (T::N - 3 * HKV) * T::C; i += blockDim.x) {
+    const int n = 3 * HKV + i / T::C, c = i % T::C;
+    *reinterpret_cast<uint16_t*>(sB + b_offset<T::N>(n, c)) = 0;
+  }
+  fence_proxy_async_smem();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDtStages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(acc_full + b, 1);
+      mbar_init(acc_empty + b, kDtTile);
+    }
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) prefetch_tmap(&tmap_v);
+  if (warp == 1) tmem_alloc(tmem_slot, T::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int gs = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+        for (int kc = 0; kc < T::kChunks; ++kc, ++gs) {
+          const int s = gs % kDtStages;
+          if (gs >= kDtStages &&
+              !mbar_wait(empty + s, ((gs / kDtStages) - 1) & 1, err, kDevErrTimeoutBase + 20)) {
+            ok = false;
+            *abort_flag = 1;
+            break;
+          }
+          if (aborted_flag(abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full + s, T::kStageBytes);
+          tma_load_2d(sA + s * T::kStageBytes, &tmap_v, full + s, kc * kDtChunk, t * kDtTile);
+        }
+      }
+      // every copy issued must land before the CTA leaves
+      for (int j = gs - kDtStages < 0 ? 0 : gs - kDtStages; j < gs; ++j)
+        mbar_wait(full + j % kDtStages, (j / kDtStages) & 1, err, kDevErrTimeoutBase + 21);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc_bf16(kDtTile, T::N, false, false);
+      const uint32_t a_lo = desc_lo(smem_u32(sA), 16), b_lo = desc_lo(smem_u32(sB), 16);
+      int gs = 0, it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++it) {
+        const int buf = it & 1;
+        if (it >= 2 && !mbar_wait_hot(acc_empty + buf, ((it - 2) >> 1) & 1, err, kDevErrTimeoutBase + 22)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + static_cast<uint32_t>(buf * T::N);
+        for (int kc = 0; kc < T::kChunks; ++kc, ++gs) {
+          const int s = gs % kDtStages;
+          if (!mbar_wait_hot(full + s, (gs / kDtStages) & 1, err, kDevErrTimeoutBase + 23)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = a_lo + static_cast<uint32_t>(s * (T::kStageBytes >> 4));
+          const uint32_t b = b_lo + static_cast<uint32_t>(kc * (T::kBChunkBytes >> 4));
+          if (kc == 0) umma_ss_w<0, kDescHiSw128, kDescHiSw128>(d, a, b, idesc);
+          else umma_ss_w<1, kDescHiSw128, kDescHiSw128>(d, a, b, idesc);
+#pragma unroll
+          for (int kk = 1; kk < 4; ++kk)
+            umma_ss_w<1, kDescHiSw128, kDescHiSw128>(d, a + 2 * kk, b + 2 * kk, idesc);
+          umma_commit(empty + s);
+        }
+        if (!ok) break;
+        umma_commit(acc_full + buf);
+      }
+      if (!ok) *abort_flag = 1;
+      umma_commit(fin);
+      mbar_wait_hot(fin, 0, err, kDevErrTimeoutBase + 24);
+    }
+    __syncwarp();
+  } else {
+    // epilogue: thread = token of the tile (TMEM lane)
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    float a[HKV];
+#pragma unroll
+    for (int g = 0; g < HKV; ++g) a[g] = A[g];
+    int it = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
+      const int buf = it & 1;
+      if (!mbar_wait(acc_full + buf, (it >> 1) & 1, err, kDevErrTimeoutBase + 25) || aborted_flag(abort_flag)) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      uint32_t r[T::N];
+      const uint32_t taddr = tmem + lane_base + static_cast<uint32_t>(buf * T::N);
+      if constexpr (T::N == 16) {
+        DMA_TMEM_LD16(taddr, r);
+      } else if constexpr (T::N == 32) {
+        DMA_TMEM_LD32(taddr, r);
+      } else {
+        DMA_TMEM_LD32(taddr, r);
+        DMA_TMEM_LD16(taddr + 32, (r + 32));
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(acc_empty + buf);
+      const long long tok = static_cast<long long>(t) * kDtTile + row;
+      if (tok < ntok) {
+        const long long b = tok / L;
+        const long long l = tok - b * L;
+#pragma unroll
+        for (int g = 0; g < HKV; ++g) {
+          const float z = (__uint_as_float(r[g]) + __uint_as_float(r[HKV + g])) + __uint_as_float(r[2 * HKV + g]);
+          dt[(b * HKV + g) * L + l] = expf(a[g] * softplus_f32(z));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, T::kTmemCols);
+}
+
+template <int HKV, int D>
+cudaError_t launch_tc(const void* v, const float* W, const float* A, long long ntok, int L, float* dt,
+                      uint32_t* err, cudaStream_t s) {
+  using T = DtTc<HKV, D>;
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap tm;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(T::C), static_cast<cuuint64_t>(ntok)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(T::C) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kDtChunk), static_cast<cuuint32_t>(kDtTile)};
+  cuuint32_t es[2] = {1, 1};
+  if (enc(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(v), dims, strides, box, es,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(dt_tc_kernel<HKV, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       T::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  int dev = 0, nsm = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return cudaErrorInvalidDevice;
+  const long long n_tiles = (ntok + kDtTile - 1) / kDtTile;
+  const int grid = static_cast<int>(n_tiles < nsm ? n_tiles : nsm);
+  dt_tc_kernel<HKV, D><<<grid, kDtTcThreads, T::kSmemBytes, s>>>(tm, W, A, static_cast<int>(ntok), L, dt, err);
+  return cudaGetLastError();
+}
 }  // namespace
 
 cudaError_t launch_dt_scores(const void* v, const float* W, const float* A, int B, int L, int Hkv, int d,
-                             float* dt, cudaStream_t s) {
+                             float* dt, uint32_t* err, cudaStream_t s) {
+  const long long ntok = static_cast<long long>(B) * L;
+  // tensor-core path: TMA needs a 16-byte aligned V and fewer than 2^31 tokens
+  if ((reinterpret_cast<uintptr_t>(v) & 15u) == 0 && ntok < (1LL << 31) && get_encode_fn()) {
+#define DMA_DT_TC(H, DD) \
+  if (Hkv == H && d == DD) return launch_tc<H, DD>(v, W, A, ntok, L, dt, err, s);
+    DMA_DT_TC(1, 64) DMA_DT_TC(2, 64) DMA_DT_TC(4, 64) DMA_DT_TC(8, 64)
+    DMA_DT_TC(1, 128) DMA_DT_TC(2, 128) DMA_DT_TC(4, 128) DMA_DT_TC(8, 128)
+#undef DMA_DT_TC
+  }
 #define DMA_DT_CASE(H, DD) \
   if (Hkv == H && d == DD) return launch_t<H, DD>(v, W, A, B, L, dt, s);
   DMA_DT_CASE(1, 64) DMA_DT_CASE(2, 64) DMA_DT_CASE(4, 64) DMA_DT_CASE(8, 64) DMA_DT_CASE(16, 64)

@@ -213,7 +213,9 @@ def time_prefill(dma, wl, steps, warmup, flush, dev, ranks_sync):
     ranks_sync()
     assert dma.dma_check(ws) == 0
     flops = prefill_flops(wl, lengths)
-    return {"flops": flops, "ms": total_ms / steps, "stage_ms": [s / steps for s in stage], "launches": 3 * steps,
+    # dt, selector (skipped when keep_window_size >= L: no top-k) and attention
+    per_step = 2 if wl.L <= wl.w else 3
+    return {"flops": flops, "ms": total_ms / steps, "stage_ms": [s / steps for s in stage], "launches": per_step * steps,
             "x": x, "ws": ws, "out": out}
 
 

@@ -330,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // work item i of this CTA: false when there is none left
   struct ItemInfo {
     Item it;
-    int nh, n_kt, n_full;
+    int nh, n_kt, n_full, n_total;
     size_t tile;
   };
   auto item_info = [&](int i, ItemInfo& x) -> bool {
@@ -339,9 +339,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     x.it = decode_item(w, npairs, Hkv, B, n_rt);
     x.nh = min(2, nrep - 2 * x.it.pair);
     x.tile = (static_cast<size_t>(x.it.b) * Hkv + x.it.g) * n_rt + x.it.t;
-    const int2 cnt = plan.counts[x.tile];
-    x.n_full = cnt.x;
-    x.n_kt = (cnt.y + kKeyTile - 1) / kKeyTile;
+    int n_total;
+    if (plan.no_topk) {
+      // keys 0 .. q in order: q = the tile's last row, or the last valid key
+      int len = plan.lengths ? plan.lengths[x.it.b] : L;
+      if (len < 1 || len > L) {
+        raise_error(err, kDevErrBadLength);
+        len = len < 1 ? 1 : L;
+      }
+      const int r0 = x.it.t * kRowTile;
+      const int q = min(r0 + min(kRowTile, L - r0) - 1, len - 1);
+      x.n_full = min(r0, q) + 1;
+      n_total = q + 1;
+    } else {
+      const int2 cnt = plan.counts[x.tile];
+      x.n_full = cnt.x;
+      n_total = cnt.y;
+    }
+    x.n_total = n_total;
+    x.n_kt = (n_total + kKeyTile - 1) / kKeyTile;
     return true;
   };
 
@@ -375,6 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t* kbase_t = plan.kbase + x.tile * (plan.cap / kKeyTile);
       const float* bias_t = plan.bias + x.tile * plan.cap;
       const uint32_t* span_t = plan.span + x.tile * plan.cap;
+      const float* dt_row = plan.dt_src + (static_cast<size_t>(x.it.b) * Hkv + g) * L;
       for (int j = 0; j < x.n_kt; ++j, ++gk) {
         const int s = gk % C::kStages;
         const int u = gk / C::kStages;
@@ -389,12 +406,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const int e = j * kKeyTile + lane * 4;
-        const int kb0 = kbase_t[j];
+        const int kb0 = plan.no_topk ? j * kKeyTile : kbase_t[j];
         {
-          const float4 bi = *reinterpret_cast<const float4*>(bias_t + e);
-          const uint4 sp = *reinterpret_cast<const uint4*>(span_t + e);
+          float bv[4];
+          uint4 sp;
+          if (plan.no_topk) {
+            // list entry e is key e; padding past the last visible key has span 0
+            const int r0 = x.it.t * kRowTile, nrows = min(kRowTile, L - r0);
+            uint32_t spv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int key = e + q;
+              const bool live = key < x.n_total;
+              bv[q] = live ? dt_row[key] : 0.0f;
+              spv[q] = live ? static_cast<uint32_t>(key > r0 ? key - r0 : 0) | (static_cast<uint32_t>(nrows) << 16)
+                            : 0u;
+            }
+            sp = make_uint4(spv[0], spv[1], spv[2], spv[3]);
+          } else {
+            const float4 bi = *reinterpret_cast<const float4*>(bias_t + e);
+            sp = *reinterpret_cast<const uint4*>(span_t + e);
+            bv[0] = bi.x; bv[1] = bi.y; bv[2] = bi.z; bv[3] = bi.w;
+          }
           *reinterpret_cast<uint4*>(sMeta + ms_slot * C::kMetaBytes + lane * 16) = sp;
-          const float bv[4] = {bi.x, bi.y, bi.z, bi.w};
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             *reinterpret_cast<uint4*>(sKx + s * kXBytes + xoff(lane * 4 + q, 0)) = bias_columns(bv[q] * inv_scale);
@@ -457,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           stop = true;
           break;
         }
-        const int kb0 = kbase_t[j];
+        const int kb0 = plan.no_topk ? j * kKeyTile : kbase_t[j];
         int4 ix = make_int4(0, 0, 0, 0);
         if (kb0 < 0) {
           ix = *reinterpret_cast<const int4*>(idx_t + j * kKeyTile + lane * 4);

@@ -95,6 +95,9 @@ PrefillPlan carve_prefill_plan(void* ws, const Geometry& g) {
   const int cap = prefill_cap(g.Lk, g.w);
   char* base = static_cast<char*>(ws);
   PrefillPlan p;
+  p.dt_src = nullptr;
+  p.lengths = nullptr;
+  p.no_topk = 0;
   size_t off = kHeaderBytes;
   p.dt = reinterpret_cast<float*>(base + off);
   off = align_up(off + bg * g.Lk * 4, 256);
@@ -244,7 +247,7 @@ dma_status_t dma_forward_prefill(const void* q, const void* k, const void* v, co
   if (ws_bytes < prefill_plan_bytes(g)) return DMA_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint32_t* err = static_cast<uint32_t*>(workspace);
-  const PrefillPlan plan = carve_prefill_plan(workspace, g);
+  PrefillPlan plan = carve_prefill_plan(workspace, g);
   cudaError_t e;
   const float* dt = dt_in;
   if ((e = stage_mark(0, s)) != cudaSuccess) return cuda_fail(e);
@@ -253,7 +256,12 @@ dma_status_t dma_forward_prefill(const void* q, const void* k, const void* v, co
     dt = plan.dt;
   }
   if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e);
-  if ((e = launch_select_prefill(dt, lengths, g, plan, err, s)) != cudaSuccess) return cuda_fail(e);
+  plan.dt_src = dt;
+  plan.lengths = lengths;
+  plan.no_topk = L <= keep_window_size;
+  // with no top-k there is nothing to select: the attention kernel derives
+  // each tile's key list (causal and padding bounds) itself
+  if (!plan.no_topk && (e = launch_select_prefill(dt, lengths, g, plan, err, s)) != cudaSuccess) return cuda_fail(e);
   if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e);
   if ((e = launch_attn_prefill(q, k, v, g, scale, plan, out, err, s)) != cudaSuccess) return cuda_fail(e);
   if ((e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e);

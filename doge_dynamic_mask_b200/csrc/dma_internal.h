@@ -54,6 +54,14 @@ struct PrefillPlan {
   int32_t* kbase;
   int cap;          // entries per tile (multiple of kKeyTile)
   int n_row_tiles;
+  // Set by the caller before the attention launch.  no_topk (Lk <= w): every
+  // row keeps every key it sees, so no list was built and the attention kernel
+  // derives each tile's list itself: keys 0 .. q in order (q the tile's last
+  // visible key, from lengths), bias dt_src[(b, g), j], key j > r0 kept from
+  // tile row j - r0 on.
+  const float* dt_src;
+  const int32_t* lengths;
+  int no_topk;
 };
 
 // Decode plan: per (batch, kv head) the kept keys in ascending index order.

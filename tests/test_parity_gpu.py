@@ -162,6 +162,9 @@ PREFILL_CASES = [
     wl(1, 1100, 6, 2, 64, 256, seed=15),
     wl(1, 1, 2, 1, 64, 4, seed=16),
     wl(1, 200, 2, 1, 128, 1, a=(-4.0, -0.1), seed=17),
+    # keep_window_size >= L: no top-k, the attention kernel builds each tile's list itself
+    wl(2, 300, 4, 2, 64, 512, lens=(150, 300), seed=18),
+    wl(3, 257, 6, 2, 128, 257, lens=(1, 129), seed=19),
 ]
 
 

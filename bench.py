@@ -251,6 +251,47 @@ def time_decode(dma, wl, steps, warmup, flush, dev, ranks_sync):
             "launches": 4 * steps}
 
 
+def time_decode_cached(dma, wl, steps, warmup, flush, dev, ranks_sync):
+    """The decode workload as incremental steps: the state is built over the
+    caches minus the last warmup + steps tokens (untimed), then every step
+    takes in one more token per sequence (dt of that token, kept-set update)
+    and attends over the kept keys."""
+    x = make_inputs(wl, device=dev)
+    start = wl.L - (warmup + steps)
+    lens = [torch.full((wl.B,), start + 1 + i, dtype=torch.int32, device=dev) for i in range(warmup + steps)]
+    state = dma.dma_decode_state_init(x["v"], x["W"], x["A"], torch.full((wl.B,), start, dtype=torch.int32,
+                                                                        device=dev), wl.w, wl.Hq)
+    assert dma.dma_check(state) == 0
+    out = torch.empty_like(x["q"])
+
+    def step(i):
+        dma.dma_decode_step_cached(x["q"], x["k"], x["v"], x["W"], x["A"], lens[i], wl.w, state, out=out)
+
+    for i in range(warmup):
+        step(i)
+        flush.zero_()
+    assert dma.dma_check(state, clear=False) == 0
+    ev = dma.StageEvents()
+    total_ms, stage = 0.0, [0.0, 0.0, 0.0]
+    ranks_sync()
+    with ev:
+        for i in range(warmup, warmup + steps):
+            step(i)
+            torch.cuda.synchronize()
+            s1, s2, s3 = ev.stage_ms()
+            total_ms += s1 + s2 + s3
+            stage = [stage[0] + s1, stage[1] + s2, stage[2] + s3]
+            flush.zero_()
+    ranks_sync()
+    assert dma.dma_check(state) == 0
+    # bytes a step must move: the new token's value row, the kept K and V rows, q and o
+    kept = min(wl.w, wl.L)
+    nbytes = wl.B * (wl.Hkv * wl.d * 2 + wl.Hkv * 2 * kept * wl.d * 2 + 2 * wl.Hq * wl.d * 2)
+    del x, state
+    return {"bytes": nbytes, "ms": total_ms / steps, "stage_ms": [s / steps for s in stage],
+            "launches": 3 * steps}
+
+
 def time_e2e(dma, wl, steps, warmup, dev):
     """Same metric through the public call with host (pinned) buffers: the H2D
     copy of every input and the D2H read of the output are inside each step."""
@@ -321,6 +362,13 @@ def run_only(args):
     if args.batch:
         wl = wl.replace(B=args.batch)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    if args.cached:
+        r = time_decode_cached(dma, wl, args.steps, args.warmup, flush, dev, torch.cuda.synchronize)
+        line = {"workload": wl.name + " (cached dt)", "B": wl.B, "value": r["bytes"] / (r["ms"] * 1e-3) / 1e9,
+                "unit": "GB/s"}
+        line.update({"ms_per_step": r["ms"], "stage_ms": r["stage_ms"], "gpu_launches": r["launches"]})
+        print(json.dumps(line), flush=True)
+        return
     if wl.mode == "prefill":
         r = time_prefill(dma, wl, args.steps, args.warmup, flush, dev, torch.cuda.synchronize)
         line = {"workload": wl.name, "B": wl.B, "value": r["flops"] / (r["ms"] * 1e-3) / 1e12, "unit": "TFLOP/s"}
@@ -410,6 +458,16 @@ def run_ours(args):
         result["gpu_launches"] += d["launches"]
         del d
         torch.cuda.empty_cache()
+        c = time_decode_cached(dma, WORKLOADS["decode"], args.steps, args.warmup, flush, dev, ranks_sync)
+        cms = rank_max(c["ms"])
+        others["decode_cached"] = {"value": round(world * c["bytes"] / (cms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                                   "ms_per_step": round(cms, 5),
+                                   "frac_of_hbm": round(c["bytes"] / (cms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                                   "bytes_per_step": c["bytes"], "stage_ms": [round(x, 5) for x in c["stage_ms"]],
+                                   "note": "incremental steps with cached dt (one new token per sequence per step)"}
+        result["gpu_launches"] += c["launches"]
+        del c
+        torch.cuda.empty_cache()
     result["workloads"] = others
 
     e2e = time_e2e(dma, wl, max(3, args.steps), args.warmup, dev)
@@ -460,6 +518,7 @@ def main():
     ap.add_argument("--quick", action="store_true", help="headline workload only")
     ap.add_argument("--only", choices=sorted(WORKLOADS), help="time one workload only (profiling)")
     ap.add_argument("--batch", type=int, default=0, help="with --only: override the batch size")
+    ap.add_argument("--cached", action="store_true", help="with --only decode: incremental steps with cached dt")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

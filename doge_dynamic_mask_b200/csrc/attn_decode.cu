@@ -71,7 +71,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const uint16_t
 #pragma unroll
   for (int s = 0; s < STEPS; ++s) {
     key_local[s] = warp * kKeysPerWarp + s * KPS + kg;
-    const int j = idx[key_local[s]];
+    // entries past the list's count are never read (key 0 stands in), so the
+    // kernel does not depend on what the rest of the list buffer holds
+    const int j = c0 + key_local[s] < count ? idx[key_local[s]] : 0;
     const size_t row = ((static_cast<size_t>(b) * Lk + j) * Hkv + g) * D + dl;
     kr[s] = __ldg(reinterpret_cast<const uint4*>(kc + row));
     vr[s] = __ldg(reinterpret_cast<const uint4*>(vc + row));

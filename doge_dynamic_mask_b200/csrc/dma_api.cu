@@ -157,6 +157,31 @@ DecodePlan carve_decode_plan(void* ws, const Geometry& g) {
 
 using namespace dma;
 
+// ---- incremental decode with cached dt -----------------------------------------
+
+namespace dma {
+// decode state = a decode plan (kept across steps) + per (b, g) the number of
+// tokens taken in and the list position of the worst kept key
+struct DecodeState {
+  DecodePlan plan;
+  int32_t* done;
+  int32_t* worst;
+};
+size_t state_extra_off(const Geometry& g) { return align_up(decode_plan_bytes(g), 256); }
+size_t state_bytes_for(const Geometry& g) {
+  const size_t bg = static_cast<size_t>(g.B) * g.Hkv;
+  return state_extra_off(g) + 2 * align_up(bg * 4, 256);
+}
+DecodeState carve_state(void* st, const Geometry& g) {
+  const size_t bg = static_cast<size_t>(g.B) * g.Hkv;
+  DecodeState s;
+  s.plan = carve_decode_plan(st, g);
+  s.done = reinterpret_cast<int32_t*>(static_cast<char*>(st) + state_extra_off(g));
+  s.worst = s.done + align_up(bg * 4, 256) / 4;
+  return s;
+}
+}  // namespace dma
+
 extern "C" {
 
 size_t dma_workspace_size(int B, int Lq, int Lk, int Hq, int Hkv, int d, int keep_window_size) {
@@ -298,6 +323,63 @@ dma_status_t dma_decode_step(const void* q, const void* k_cache, const void* v_c
   if ((e = launch_select_decode(dt, lengths, g, plan, err, s)) != cudaSuccess) return cuda_fail(e);
   if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e);
   if ((e = launch_attn_decode(q, k_cache, v_cache, g, scale, plan, out, s)) != cudaSuccess) return cuda_fail(e);
+  if ((e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e);
+  return DMA_OK;
+}
+
+
+size_t dma_decode_state_size(int B, int Lk, int Hq, int Hkv, int d, int keep_window_size) {
+  if (check_shape(B, Lk, Hq, Hkv, d, keep_window_size) != DMA_OK) return 0;
+  return dma::state_bytes_for(Geometry{B, 1, Lk, Hq, Hkv, d, keep_window_size});
+}
+
+dma_status_t dma_decode_state_init(const void* v_cache, const float* W_dt, const float* A, const int32_t* lengths,
+                                   int B, int Lk, int Hq, int Hkv, int d, int keep_window_size, void* state,
+                                   size_t state_bytes, dma_stream_t stream) {
+  if (!v_cache || !W_dt || !A || !state) return DMA_ERR_INVALID_ARG;
+  if (!aligned16(v_cache) || !aligned16(W_dt) || !aligned16(A) || !aligned16(state) ||
+      (lengths && !aligned16(lengths)))
+    return DMA_ERR_INVALID_ARG;
+  dma_status_t st = check_shape(B, Lk, Hq, Hkv, d, keep_window_size);
+  if (st != DMA_OK) return st;
+  if ((st = device_ok()) != DMA_OK) return st;
+  const Geometry g{B, 1, Lk, Hq, Hkv, d, keep_window_size};
+  if (state_bytes < dma::state_bytes_for(g)) return DMA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t* err = static_cast<uint32_t*>(state);
+  const dma::DecodeState ds = dma::carve_state(state, g);
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(state, 0, kHeaderBytes, s)) != cudaSuccess) return cuda_fail(e);
+  if ((e = launch_dt_scores(v_cache, W_dt, A, B, Lk, Hkv, d, ds.plan.dt, err, s)) != cudaSuccess) return cuda_fail(e);
+  if ((e = launch_select_decode(ds.plan.dt, lengths, g, ds.plan, err, s)) != cudaSuccess) return cuda_fail(e);
+  if ((e = launch_decode_state_finish(lengths, g, ds.plan, ds.done, ds.worst, s)) != cudaSuccess) return cuda_fail(e);
+  return DMA_OK;
+}
+
+dma_status_t dma_decode_step_cached(const void* q, const void* k_cache, const void* v_cache, const float* W_dt,
+                                    const float* A, const int32_t* lengths, int B, int Lk, int Hq, int Hkv, int d,
+                                    int keep_window_size, float scale, void* out, void* state, size_t state_bytes,
+                                    dma_stream_t stream) {
+  if (!q || !k_cache || !v_cache || !W_dt || !A || !out || !state) return DMA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned16(state) ||
+      !aligned16(W_dt) || !aligned16(A) || (lengths && !aligned16(lengths)))
+    return DMA_ERR_INVALID_ARG;
+  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return DMA_ERR_INVALID_ARG;
+  dma_status_t st = check_shape(B, Lk, Hq, Hkv, d, keep_window_size);
+  if (st != DMA_OK) return st;
+  if ((st = device_ok()) != DMA_OK) return st;
+  const Geometry g{B, 1, Lk, Hq, Hkv, d, keep_window_size};
+  if (state_bytes < dma::state_bytes_for(g)) return DMA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t* err = static_cast<uint32_t*>(state);
+  const dma::DecodeState ds = dma::carve_state(state, g);
+  cudaError_t e;
+  if ((e = stage_mark(0, s)) != cudaSuccess) return cuda_fail(e);
+  if ((e = launch_decode_update(v_cache, W_dt, A, lengths, g, ds.plan, ds.done, ds.worst, err, s)) != cudaSuccess)
+    return cuda_fail(e);
+  if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e);
+  if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e);
+  if ((e = launch_attn_decode(q, k_cache, v_cache, g, scale, ds.plan, out, s)) != cudaSuccess) return cuda_fail(e);
   if ((e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e);
   return DMA_OK;
 }

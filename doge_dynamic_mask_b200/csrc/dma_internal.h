@@ -105,5 +105,11 @@ cudaError_t launch_attn_prefill(const void* q, const void* k, const void* v, con
                                 const PrefillPlan& plan, void* out, uint32_t* err, cudaStream_t s);
 cudaError_t launch_attn_decode(const void* q, const void* k, const void* v, const Geometry& g, float scale,
                                const DecodePlan& plan, void* out, cudaStream_t s);
+// incremental decode: take in the tokens cached since the last step / finish a freshly selected state
+cudaError_t launch_decode_update(const void* v_cache, const float* W, const float* A, const int32_t* lengths,
+                                 const Geometry& g, const DecodePlan& plan, int32_t* done, int32_t* worst,
+                                 uint32_t* err, cudaStream_t s);
+cudaError_t launch_decode_state_finish(const int32_t* lengths, const Geometry& g, const DecodePlan& plan,
+                                       int32_t* done, int32_t* worst, cudaStream_t s);
 
 }  // namespace dma

@@ -36,6 +36,12 @@ _lib.dma_forward_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _
                                      _vp]
 _lib.dma_decode_step.restype = _i
 _lib.dma_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _sz, _vp]
+_lib.dma_decode_state_size.restype = _sz
+_lib.dma_decode_state_size.argtypes = [_i] * 6
+_lib.dma_decode_state_init.restype = _i
+_lib.dma_decode_state_init.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
+_lib.dma_decode_step_cached.restype = _i
+_lib.dma_decode_step_cached.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _sz, _vp]
 _lib.dma_check.restype = _i
 _lib.dma_check.argtypes = [_vp, _i, _vp]
 _lib.dma_status_string.restype = ctypes.c_char_p
@@ -137,6 +143,59 @@ def dma_decode_step(q, k_cache, v_cache, W_dt, A, lengths, keep_window_size, sca
                              workspace.numel(), _stream(stream)),
         "dma_decode_step")
     return out
+
+
+def dma_decode_state_size(B, Lk, Hq, Hkv, d, keep_window_size) -> int:
+    return int(_lib.dma_decode_state_size(B, Lk, Hq, Hkv, d, keep_window_size))
+
+
+def dma_decode_state_init(v_cache, W_dt, A, lengths, keep_window_size, Hq, state=None, stream=None):
+    """Decode state for incremental steps: dt of every cached token and each
+    (batch, kv head)'s kept set.  Returns the state (a uint8 device tensor)."""
+    B, Lk, Hkv, d = v_cache.shape
+    size = dma_decode_state_size(B, Lk, Hq, Hkv, d, keep_window_size)
+    if size == 0:
+        raise ValueError("unsupported decode geometry")
+    if state is None:
+        state = torch.empty(size, dtype=torch.uint8, device=v_cache.device)
+    _ok(_lib.dma_decode_state_init(_ptr(v_cache), _ptr(W_dt), _ptr(A), _ptr(lengths), B, Lk, Hq, Hkv, d,
+                                   keep_window_size, _ptr(state), state.numel(), _stream(stream)),
+        "dma_decode_state_init")
+    return state
+
+
+def dma_decode_step_cached(q, k_cache, v_cache, W_dt, A, lengths, keep_window_size, state, scale=None, out=None,
+                           stream=None):
+    """One decode step that takes in only the tokens cached since the previous step."""
+    B, Hq, d = q.shape
+    Lk, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    _ok(_lib.dma_decode_step_cached(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(W_dt), _ptr(A), _ptr(lengths), B,
+                                    Lk, Hq, Hkv, d, keep_window_size, float(scale), _ptr(out), _ptr(state),
+                                    state.numel(), _stream(stream)),
+        "dma_decode_step_cached")
+    return out
+
+
+def decode_state_views(state, B, Lk, Hq, Hkv, d, keep_window_size):
+    """(dt [B, Hkv, Lk] float32, kept count [B, Hkv] int32, kept key lists [B, Hkv, cap] int32) views of a
+    decode state, for tests: the layout is that of a decode workspace."""
+    bg = B * Hkv
+    cap = -(-min(Lk, keep_window_size) // 128) * 128
+    def up(x):
+        return -(-x // 256) * 256
+    off = 256
+    dt = state[off:off + bg * Lk * 4].view(torch.float32).view(B, Hkv, Lk)
+    off = up(off + bg * Lk * 4)
+    off = up(off + bg * 8)                   # tau
+    idx = state[off:off + bg * cap * 4].view(torch.int32).view(B, Hkv, cap)
+    off = up(off + bg * cap * 4)
+    off = up(off + bg * cap * 4)             # bias
+    count = state[off:off + bg * 4].view(torch.int32).view(B, Hkv)
+    return dt, count, idx
 
 
 def dma_check(workspace, clear=True, stream=None) -> int:

@@ -130,6 +130,44 @@ DMA_API dma_status_t dma_decode_step(const void* q, const void* k_cache, const v
                              size_t ws_bytes, dma_stream_t stream);
 
 /*
+ * Incremental decode with cached dt.  dt is one linear projection per cached
+ * token followed by exp(A * softplus(.)) ([DMA step 3]), so a token's dt never
+ * changes once it is cached: this pair of calls keeps dt and each (b, g)'s
+ * kept set in a caller-owned decode state and, per step, takes in only the
+ * tokens cached since the previous step (compute their dt; append while fewer
+ * than keep_window_size keys are kept, else replace the worst kept key when
+ * the new one ranks higher).  The output of a step equals dma_decode_step's
+ * for the same caches and lengths; the per-step cost no longer includes the
+ * scan of the whole value cache.
+ *
+ *   dma_decode_state_size  bytes of a decode state for this geometry (0 when
+ *                          unsupported, as dma_workspace_size).
+ *   dma_decode_state_init  dt over every cached token (lengths[b] of them) and
+ *                          the full top-keep_window_size selection; clears the
+ *                          state's status word.  The state (16-byte aligned
+ *                          device memory, state_bytes >= the size above)
+ *                          then belongs to these calls until the caller frees
+ *                          it; dma_check(state) reports its status word.
+ *   dma_decode_step_cached  one decode step: lengths[b] may grow by any number
+ *                          of tokens since the previous call (the new tokens'
+ *                          K and V already in the caches); a length outside
+ *                          [1, Lk] or below the previous one is reported as
+ *                          DMA_ERR_BAD_LENGTH through dma_check and that
+ *                          sequence's state is left unchanged.  Arguments
+ *                          as dma_decode_step.  Calls on one state must be
+ *                          ordered (one stream).
+ */
+DMA_API size_t dma_decode_state_size(int B, int Lk, int Hq, int Hkv, int d, int keep_window_size);
+DMA_API dma_status_t dma_decode_state_init(const void* v_cache, const float* W_dt, const float* A,
+                                           const int32_t* lengths, int B, int Lk, int Hq, int Hkv, int d,
+                                           int keep_window_size, void* state, size_t state_bytes,
+                                           dma_stream_t stream);
+DMA_API dma_status_t dma_decode_step_cached(const void* q, const void* k_cache, const void* v_cache,
+                                            const float* W_dt, const float* A, const int32_t* lengths, int B,
+                                            int Lk, int Hq, int Hkv, int d, int keep_window_size, float scale,
+                                            void* out, void* state, size_t state_bytes, dma_stream_t stream);
+
+/*
  * dma_decode_step without a caller-provided workspace (the pages have no
  * counterpart: this is a calling convention of this library).
  *

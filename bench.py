@@ -294,31 +294,57 @@ def time_decode_cached(dma, wl, steps, warmup, flush, dev, ranks_sync):
 
 def time_e2e(dma, wl, steps, warmup, dev):
     """Same metric through the public call with host (pinned) buffers: the H2D
-    copy of every input and the D2H read of the output are inside each step."""
+    copy of every input and the D2H read of the output are inside each step.
+    Steps are pipelined as a serving loop would run them: step i+1's inputs
+    travel host-to-device (one stream) while step i computes (a second) and
+    step i-1's output travels device-to-host (a third), with two device
+    copies of the inputs and the output; every step still copies its own
+    inputs in and its own result out."""
     xh = {k: v.pin_memory() for k, v in make_inputs(wl, device="cpu").items()}
     lengths = xh["lengths"].numpy()
-    xd = {k: torch.empty_like(v, device=dev) for k, v in xh.items()}
-    ws = dma.new_workspace(dma.dma_workspace_size(wl.B, wl.L, wl.L, wl.Hq, wl.Hkv, wl.d, wl.w), dev)
-    out_d = torch.empty_like(xd["q"])
-    out_h = torch.empty_like(xh["q"]).pin_memory()
+    xd = [{k: torch.empty_like(v, device=dev) for k, v in xh.items()} for _ in range(2)]
+    ws = [dma.new_workspace(dma.dma_workspace_size(wl.B, wl.L, wl.L, wl.Hq, wl.Hkv, wl.d, wl.w), dev)
+          for _ in range(2)]
+    out_d = [torch.empty_like(xd[0]["q"]) for _ in range(2)]
+    out_h = [torch.empty_like(xh["q"]).pin_memory() for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in xh.values())
-    d2h = out_h.numel() * out_h.element_size()
+    d2h = out_h[0].numel() * out_h[0].element_size()
+    s_in, s_comp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    started = [False, False]
 
-    def step():
-        for k in xh:
-            xd[k].copy_(xh[k], non_blocking=True)
-        dma.dma_forward_prefill(xd["q"], xd["k"], xd["v"], xd["W"], xd["A"], xd["lengths"], wl.w, out=out_d,
-                                workspace=ws)
-        out_h.copy_(out_d, non_blocking=True)
+    def step(i):
+        k = i & 1
+        with torch.cuda.stream(s_in):
+            if started[k]:
+                s_in.wait_event(ev_comp[k])          # step i-2 has read these inputs
+            for name in xh:
+                xd[k][name].copy_(xh[name], non_blocking=True)
+            ev_in[k].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(ev_in[k])
+            if started[k]:
+                s_comp.wait_event(ev_out[k])         # step i-2's output has left
+            dma.dma_forward_prefill(xd[k]["q"], xd[k]["k"], xd[k]["v"], xd[k]["W"], xd[k]["A"], xd[k]["lengths"],
+                                    wl.w, out=out_d[k], workspace=ws[k])
+            ev_comp[k].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[k])
+            out_h[k].copy_(out_d[k], non_blocking=True)
+            ev_out[k].record(s_out)
+        started[k] = True
 
-    for _ in range(warmup):
-        step()
+    for i in range(warmup):
+        step(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        step()
-    e1.record()
+    e0.record(s_in)
+    for i in range(warmup, warmup + steps):
+        step(i)
+    s_in.wait_stream(s_out)
+    e1.record(s_in)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     return {"tflops": prefill_flops(wl, lengths) / (ms * 1e-3) / 1e12, "ms": ms, "h2d": h2d, "d2h": d2h}

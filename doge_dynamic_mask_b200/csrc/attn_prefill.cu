@@ -62,7 +62,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 // every kPolyEvery-th pair of probabilities in a row is computed on the FMA pipe
 // (exp2_poly_x2), the rest on the MUFU
-constexpr int kPolyEvery = 4;
+constexpr int kPolyEvery = 5;
 constexpr int kXBytes = kKeyTile * 32;       // 128 rows x 16 bf16 extra K columns (bias / ones)
 
 template <int D>

@@ -93,3 +93,40 @@ def test_argument_errors_are_reported_before_any_device_work(lib):
     lib.dma_dt_scores.argtypes = [vp, vp, vp] + [ctypes.c_int] * 4 + [vp, vp]
     assert lib.dma_dt_scores(p16, p16, p16, 1, 16, 3, 64, p16, None) == 2          # Hkv = 3
     assert lib.dma_dt_scores(p16, p16, p16, 0, 16, 2, 64, p16, None) == 1          # B = 0
+
+
+def test_cached_decode_state_size_and_argument_errors(lib):
+    vp = ctypes.c_void_p
+    p16 = vp(1 << 20)          # aligned dummy address, never dereferenced
+    bad = vp((1 << 20) + 4)    # misaligned
+    size = lib.dma_decode_state_size
+    size.restype = ctypes.c_size_t
+    size.argtypes = [ctypes.c_int] * 6
+    ws = lib.dma_workspace_size
+    ws.restype = ctypes.c_size_t
+    # a state holds a decode workspace's plan plus two ints per (batch, kv head)
+    assert size(64, 65536, 16, 8, 128, 2048) >= ws(64, 1, 65536, 16, 8, 128, 2048) + 2 * 64 * 8 * 4
+    assert size(1, 256, 6, 4, 64, 64) == 0          # Hq not a multiple of Hkv
+    assert size(1, 256, 4, 2, 96, 64) == 0          # d not supported
+    init = lib.dma_decode_state_init
+    init.restype = ctypes.c_int
+    init.argtypes = [vp, vp, vp, vp] + [ctypes.c_int] * 6 + [vp, ctypes.c_size_t, vp]
+    args = [p16, p16, p16, None, 1, 256, 4, 2, 64, 64, p16, 1 << 30, None]
+    a = list(args); a[0] = None
+    assert init(*a) == 1
+    a = list(args); a[10] = bad
+    assert init(*a) == 1
+    a = list(args); a[8] = 80
+    assert init(*a) == 2                             # DMA_ERR_UNSUPPORTED
+    step = lib.dma_decode_step_cached
+    step.restype = ctypes.c_int
+    step.argtypes = [vp, vp, vp, vp, vp, vp] + [ctypes.c_int] * 6 + [ctypes.c_float, vp, vp, ctypes.c_size_t, vp]
+    args = [p16, p16, p16, p16, p16, None, 1, 256, 4, 2, 64, 64, 0.125, p16, p16, 1 << 30, None]
+    a = list(args); a[14] = None                     # no state
+    assert step(*a) == 1
+    a = list(args); a[3] = None                      # W is required: the step computes dt of new tokens
+    assert step(*a) == 1
+    a = list(args); a[12] = float("nan")
+    assert step(*a) == 1
+    a = list(args); a[8] = 6; a[9] = 4
+    assert step(*a) == 1

@@ -5,38 +5,47 @@
 // head_dim^-0.5 plus the additive dynamic mask (dt on kept keys, min_dtype
 // elsewhere), softmax in float32, times V.
 //
-// Design.  One CTA per (row tile of 128 queries, pair of query heads of one kv
-// group).  The selector's list for the row tile names the at most
-// w + 127 keys any of its rows keeps; the kernel streams those keys in tiles of
-// 128 and never touches a key the tile does not keep.
-//   * warp 0 (K producer): TMA loads the two Q tiles once; for every key tile
-//     it fetches the 128 listed K rows into a ring of shared-memory stages
-//     (128-byte swizzle): one box copy per 64-column slab when the listed keys
-//     are one ascending run, else tile::gather4 (four listed rows per
-//     instruction).  It also writes the tile's bias columns (below) and row
-//     intervals.
-//   * warp 2 (V producer): the same for V, on its own ring release, so a slow
-//     V stage never holds back the next K tile.
-//   * warp 1: allocates the 512 TMEM columns (S_0, S_1, O_0, O_1, and at
-//     d = 64 also P_0, P_1) and, one thread, issues tcgen05.mma.  S_h = Q_h K^T (M=128, N=128, K=d) plus one
-//     more K=16 step that adds the dt bias: Q gets three columns of ones and
-//     each key row three columns holding dt/scale split into three bf16 terms
-//     (hi + mid + lo reproduce the float32 value; products with 1 are exact and
-//     the tensor core accumulates in float32), so S_h * scale = scale q.k + dt.
+// Design.  A work item is a row tile of 128 queries and a pair of query heads
+// of one kv group.  The selector's list for the row tile names the at most
+// w + 127 keys any of its rows keeps (or, without top-k, the kernel derives
+// the list itself: the keys up to the tile's last visible row); the kernel
+// streams those keys in tiles of 128 and never touches a key the tile does
+// not keep.  The kernel is persistent: one CTA per SM walks a snake order over
+// the work items (heaviest row tiles first), and every role counts key tiles
+// across items so rings and barrier phases carry on from item to item.
+// 384 threads in three warpgroups:
+//   * warp 0 (K producer): TMA loads the item's Q tiles (after the previous
+//     item's last Q K^T, signalled by q_empty); for every key tile it fetches
+//     the 128 listed K rows into a ring of shared-memory stages (128-byte
+//     swizzle): one box copy per 64-column slab when the listed keys are one
+//     ascending run, else tile::gather4 (four listed rows per instruction).
+//     It also writes the tile's bias columns (below) and row intervals.
+//   * warp 2 (V producer): the same for V, on its own ring release.
+//   * warp 1: allocates the 512 TMEM columns and, one thread, issues
+//     tcgen05.mma from 32-bit descriptor low words (the high words are
+//     constants).  S_h = Q_h K^T (M=128, N=128, K=d) plus one more K=16 step
+//     that adds the dt bias: Q gets three columns of ones and each key row
+//     three columns holding dt/scale split into three bf16 terms (hi + mid +
+//     lo reproduce the float32 value; products with 1 are exact and the tensor
+//     core accumulates in float32), so S_h * scale = scale q.k + dt.
 //     O_h += P_h V with A = P read from TMEM and B = V from shared memory.
-//     At d = 64, P has its own TMEM columns: the softmax releases S as soon as
-//     it has read it, so QK_h(j+1) runs during the softmax of tile j.  At
-//     d = 128 P is written over S and the order per key tile is PV_0(j),
-//     QK_0(j+1), PV_1(j), QK_1(j+1): while one head's softmax runs the tensor
-//     core works for the other head.
-//   * warps 3-6 / 7-10 (softmax, one thread per query row; four consecutive
-//     warps cover the four TMEM lane quarters): read S from TMEM, mask rows
-//     outside a key's row interval on the few tiles not kept by every row,
-//     take the row max of the raw scores, and form p = 2^(S*scale*log2e - m)
-//     with packed f32x2 arithmetic; P goes back over S in TMEM as bf16.  O is
-//     rescaled only when the running max grew by more than 2^8 (exact: the
-//     final division uses the same stale max).
-//   * epilogue: O / l in float32, rounded to bf16.
+//     d = 64 (S_0 S_1 O_0 O_1 P_0 P_1): the two heads run in lockstep with
+//     interleaved MMAs; QK(j+1) is issued as soon as the softmax has read
+//     S(j) and runs during the softmax of tile j.  d = 128 (P written over S):
+//     fixed ping-pong order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so the
+//     tensor core works for one head while the other head's softmax runs.
+//     Warpgroup 0 gives registers back (setmaxnreg.dec) to the softmax
+//     warpgroups (setmaxnreg.inc).
+//   * warpgroups 1 and 2 (softmax, one per head of the pair, one thread per
+//     query row; four consecutive warps cover the four TMEM lane quarters):
+//     read S from TMEM, mask rows outside a key's row interval on the few
+//     tiles not kept by every row, take the row max of the raw scores, and form
+//     p = 2^(S*scale*log2e - m) with packed f32x2 arithmetic (a fixed share of
+//     the pairs by a cubic on the FMA pipe, the rest by the MUFU ex2); P goes
+//     to TMEM as bf16.  O is rescaled only when the running max grew by more
+//     than 2^8 (exact: the final division uses the same stale max).  After
+//     the item's last tile they write O / l in float32, rounded to bf16, while
+//     the next item's first Q K^T already runs.
 // Every wait is bounded; a wait that gives up records an error and the CTA
 // drains its in-flight copies and MMAs before it frees TMEM and exits.
 #include <cuda.h>

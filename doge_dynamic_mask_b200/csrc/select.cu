@@ -7,21 +7,25 @@
 // positions of each row survive).  Causal masking is merged before the top-k,
 // ties go to the lower key index.
 //
-// Prefill (one CTA per (batch, kv head, 128-row tile)).  dt does not depend on
-// the query, so the row threshold tau_i (the composite key of row i's worst
-// kept key) never decreases along the rows: each key is kept on one contiguous
-// interval of rows, and the union of the kept sets of a row tile is the w keys
-// kept at its first row plus at most 127 newer keys.  The CTA
-//   1. radix-selects tau at the tile's first row over the keys it sees,
+// Prefill (one CTA per (batch, kv head, run of consecutive 128-row tiles)).
+// dt does not depend on the query, so the row threshold tau_i (the composite
+// key of row i's worst kept key) never decreases along the rows: each key is
+// kept on one contiguous interval of rows, and the union of the kept sets of a
+// row tile is the w keys kept at its first row plus at most 127 newer keys.
+// For each tile of its run the CTA
+//   1. finds tau at the tile's first row: by radix selection over the keys
+//      that row sees (the run's first tile), or from the previous tile's
+//      last-row kept set plus at most one new key (every later tile),
 //   2. collects the union U (keys <= the tile's last visible row whose key is
-//      >= that tau) in index order,
+//      >= that tau) in index order: from the prefix in global memory, or from
+//      the previous tile's union and the tile's own new keys,
 //   3. takes the 128 smallest keys of U, in which every later row's tau lies,
 //      and resolves tau_i for each row of the tile,
 //   4. gives each key of U its row interval [lo, hi) inside the tile and writes
 //      the list: keys kept by every row first, then the rest (index order in
 //      each class), each with its dt bias and interval.
-// Tiles whose rows see at most w keys (and every tile when Lk <= w) keep every
-// visible key and skip the selection.
+// Tiles whose rows see at most w keys (and every tile when Lk <= w) keep
+// every visible key and skip the selection.
 //
 // Decode (one CTA per (batch, kv head)): the single query at len_b - 1 keeps
 // the w best of its len_b keys; radix-select the w-th key, then compact the

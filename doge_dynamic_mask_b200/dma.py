@@ -42,6 +42,8 @@ _lib.dma_decode_state_init.restype = _i
 _lib.dma_decode_state_init.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
 _lib.dma_decode_step_cached.restype = _i
 _lib.dma_decode_step_cached.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _sz, _vp]
+_lib.dma_selftest_wait.restype = _i
+_lib.dma_selftest_wait.argtypes = [_vp, _vp]
 _lib.dma_check.restype = _i
 _lib.dma_check.argtypes = [_vp, _i, _vp]
 _lib.dma_status_string.restype = ctypes.c_char_p
@@ -196,6 +198,12 @@ def decode_state_views(state, B, Lk, Hq, Hkv, d, keep_window_size):
     off = up(off + bg * cap * 4)             # bias
     count = state[off:off + bg * 4].view(torch.int32).view(B, Hkv)
     return dt, count, idx
+
+
+def dma_selftest_wait(workspace, stream=None):
+    """Launch the bounded-wait diagnostic: its wait runs out (about one second)
+    and records a timeout that dma_check then reports."""
+    _ok(_lib.dma_selftest_wait(_ptr(workspace), _stream(stream)), "dma_selftest_wait")
 
 
 def dma_check(workspace, clear=True, stream=None) -> int:

@@ -213,6 +213,16 @@ DMA_API dma_status_t dma_check(void* workspace, int clear, dma_stream_t stream);
  */
 DMA_API dma_status_t dma_set_stage_events(void* const* events, int n);
 
+/*
+ * Diagnostic (no counterpart on the pages): exercises the bounded-wait path
+ * every kernel of this library uses.  One device thread waits on a barrier
+ * that nothing completes; after the library's wait limit (about one second)
+ * it gives up and records a timeout in the workspace's status word, which
+ * dma_check() then reports as DMA_ERR_TIMEOUT.  workspace: at least 256
+ * bytes, 16-byte aligned, zeroed before use.  Nothing faults or hangs.
+ */
+DMA_API dma_status_t dma_selftest_wait(void* workspace, dma_stream_t stream);
+
 /* Human-readable name of a status. Never NULL. */
 DMA_API const char* dma_status_string(dma_status_t status);
 

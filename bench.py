@@ -9,9 +9,12 @@ call (dt scores, dynamic-mask selection, attention).  The same line reports
 decode GB/s (B=64, cache 65536, Hq=16, Hkv=8, d=128, w=2048; algorithmic KV
 bytes) and TFLOP/s of the sparse-padded and long-context prefill workloads.
 
-Timing: CUDA events per step on the launching stream, L2 flushed (256 MiB
-write) between timed steps, W untimed warm-up steps, a barrier and a device
-synchronize on both sides of the timed region, max over ranks.  Multi-GPU:
+Timing: a CUDA event pair per step on the launching stream, L2 flushed
+(256 MiB write) between timed steps, the K timed steps enqueued ahead of the
+device so that no host gap is timed, W untimed warm-up steps, a barrier and a
+device synchronize on both sides of the timed region, max over ranks.  The
+stage split (and the attention kernel's time for the roofline) comes from K
+more steps after the timed region, each with the library's stage events.  Multi-GPU:
 one process per GPU (torchrun), every rank runs its own copy of the workload
 (weak scaling, no data-path collective).
 
@@ -186,6 +189,51 @@ def cpu_cores():
 # our arm
 # ----------------------------------------------------------------------------
 
+def run_steps(dma, step, first, steps, flush, stages=False):
+    """Device time of `steps` calls step(first), step(first + 1), ...: the L2
+    flush runs between calls, and all of it is enqueued before one
+    synchronize, with a few flushes queued ahead of the first call so that
+    the host enqueues ahead of the device: the events time device work only,
+    never a host gap.  Without `stages` one event pair brackets each call and
+    the per-call milliseconds are returned.  With `stages` every call records
+    the library's four stage events (before S1, after S1, after S2, after the
+    attention) and the per-call (S1, S2, attention) milliseconds are
+    returned; an event waits for the work before it, so the two events
+    inside the call add a little device time (about 2.5 us each) and this
+    pass gives the split, not the step time."""
+    torch.cuda.synchronize()
+    if stages:
+        evs = [dma.StageEvents() for _ in range(steps)]
+    else:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for _ in range(4):
+        flush.zero_()
+    for i, ev in enumerate(evs):
+        if stages:
+            with ev:
+                step(first + i)
+        else:
+            ev[0].record()
+            step(first + i)
+            ev[1].record()
+        flush.zero_()
+    torch.cuda.synchronize()
+    if stages:
+        return [ev.stage_ms() for ev in evs]
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def timed(dma, step, first, steps, flush, ranks_sync):
+    """The timed region (barrier + synchronize on both sides) and, after it,
+    the stage-split pass: (ms per step, [S1, S2, attention] ms per step)."""
+    ranks_sync()
+    ms = run_steps(dma, step, first, steps, flush)
+    ranks_sync()
+    split = run_steps(dma, step, first + steps, steps, flush, stages=True)
+    n = len(split)
+    return sum(ms) / len(ms), [sum(x[k] for x in split) / n for k in range(3)]
+
+
 def time_prefill(dma, wl, steps, warmup, flush, dev, ranks_sync):
     x = make_inputs(wl, device=dev)
     lengths = x["lengths"].cpu().numpy()
@@ -199,23 +247,12 @@ def time_prefill(dma, wl, steps, warmup, flush, dev, ranks_sync):
         step()
         flush.zero_()
     assert dma.dma_check(ws) == 0
-    ev = dma.StageEvents()
-    total_ms, stage = 0.0, [0.0, 0.0, 0.0]
-    ranks_sync()
-    with ev:
-        for _ in range(steps):
-            step()
-            torch.cuda.synchronize()
-            s1, s2, s3 = ev.stage_ms()
-            total_ms += s1 + s2 + s3
-            stage = [stage[0] + s1, stage[1] + s2, stage[2] + s3]
-            flush.zero_()
-    ranks_sync()
+    ms, stage = timed(dma, lambda i: step(), 0, steps, flush, ranks_sync)
     assert dma.dma_check(ws) == 0
     flops = prefill_flops(wl, lengths)
     # dt, selector (skipped when keep_window_size >= L: no top-k) and attention
     per_step = 2 if wl.L <= wl.w else 3
-    return {"flops": flops, "ms": total_ms / steps, "stage_ms": [s / steps for s in stage], "launches": per_step * steps,
+    return {"flops": flops, "ms": ms, "stage_ms": stage, "launches": per_step * steps,
             "x": x, "ws": ws, "out": out}
 
 
@@ -232,33 +269,22 @@ def time_decode(dma, wl, steps, warmup, flush, dev, ranks_sync):
         step()
         flush.zero_()
     assert dma.dma_check(ws) == 0
-    ev = dma.StageEvents()
-    total_ms, stage = 0.0, [0.0, 0.0, 0.0]
-    ranks_sync()
-    with ev:
-        for _ in range(steps):
-            step()
-            torch.cuda.synchronize()
-            s1, s2, s3 = ev.stage_ms()
-            total_ms += s1 + s2 + s3
-            stage = [stage[0] + s1, stage[1] + s2, stage[2] + s3]
-            flush.zero_()
-    ranks_sync()
+    ms, stage = timed(dma, lambda i: step(), 0, steps, flush, ranks_sync)
     assert dma.dma_check(ws) == 0
     nbytes = decode_bytes(wl, lengths)
     del x
-    return {"bytes": nbytes, "ms": total_ms / steps, "stage_ms": [s / steps for s in stage],
-            "launches": 4 * steps}
+    return {"bytes": nbytes, "ms": ms, "stage_ms": stage, "launches": 4 * steps}
 
 
 def time_decode_cached(dma, wl, steps, warmup, flush, dev, ranks_sync):
     """The decode workload as incremental steps: the state is built over the
-    caches minus the last warmup + steps tokens (untimed), then every step
+    caches minus the last warmup + 2 * steps tokens (untimed), then every step
     takes in one more token per sequence (dt of that token, kept-set update)
     and attends over the kept keys."""
     x = make_inputs(wl, device=dev)
-    start = wl.L - (warmup + steps)
-    lens = [torch.full((wl.B,), start + 1 + i, dtype=torch.int32, device=dev) for i in range(warmup + steps)]
+    n_calls = warmup + 2 * steps   # warm-up, timed steps, stage-split steps
+    start = wl.L - n_calls
+    lens = [torch.full((wl.B,), start + 1 + i, dtype=torch.int32, device=dev) for i in range(n_calls)]
     state = dma.dma_decode_state_init(x["v"], x["W"], x["A"], torch.full((wl.B,), start, dtype=torch.int32,
                                                                         device=dev), wl.w, wl.Hq)
     assert dma.dma_check(state) == 0
@@ -271,25 +297,13 @@ def time_decode_cached(dma, wl, steps, warmup, flush, dev, ranks_sync):
         step(i)
         flush.zero_()
     assert dma.dma_check(state, clear=False) == 0
-    ev = dma.StageEvents()
-    total_ms, stage = 0.0, [0.0, 0.0, 0.0]
-    ranks_sync()
-    with ev:
-        for i in range(warmup, warmup + steps):
-            step(i)
-            torch.cuda.synchronize()
-            s1, s2, s3 = ev.stage_ms()
-            total_ms += s1 + s2 + s3
-            stage = [stage[0] + s1, stage[1] + s2, stage[2] + s3]
-            flush.zero_()
-    ranks_sync()
+    ms, stage = timed(dma, step, warmup, steps, flush, ranks_sync)
     assert dma.dma_check(state) == 0
     # bytes a step must move: the new token's value row, the kept K and V rows, q and o
     kept = min(wl.w, wl.L)
     nbytes = wl.B * (wl.Hkv * wl.d * 2 + wl.Hkv * 2 * kept * wl.d * 2 + 2 * wl.Hq * wl.d * 2)
     del x, state
-    return {"bytes": nbytes, "ms": total_ms / steps, "stage_ms": [s / steps for s in stage],
-            "launches": 3 * steps}
+    return {"bytes": nbytes, "ms": ms, "stage_ms": stage, "launches": 3 * steps}
 
 
 def time_e2e(dma, wl, steps, warmup, dev):

@@ -302,9 +302,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < C::kMetaSlots; ++s) mbar_init(bars.meta_full + s, 1);
     for (int h = 0; h < 2; ++h) {
       mbar_init(bars.s_full + h, 1);
-      // the lockstep (separate-P) layout uses index 0 for both heads
-      mbar_init(bars.s_free + h, C::kSepP ? hw * kRowTile : kRowTile);
-      mbar_init(bars.p_ready + h, C::kSepP ? hw * kRowTile : kRowTile);
+      // the lockstep (separate-P) layout uses index 0 for both heads; one
+      // arrival per softmax warp (four per head)
+      mbar_init(bars.s_free + h, C::kSepP ? hw * 4 : 4);
+      mbar_init(bars.p_ready + h, C::kSepP ? hw * 4 : 4);
       mbar_init(bars.o_done + h, 1);
     }
     mbar_init(bars.fin, 1);
@@ -680,11 +681,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; ok && j < n_kt; ++j) {
             const int gt = g + j;
             ok = mbar_wait(bars.s_full, gt & 1, err, kDevErrTimeoutBase + 10) && !aborted(abort_flag);
-            if (!ok) break;
-            mbar_arrive(bars.s_free);
+            if (!(ok = __all_sync(0xFFFFFFFFu, ok))) break;
+            mbar_arrive_warp(bars.s_free);
             if (j > 0) ok = mbar_wait(bars.o_done, (gt - 1) & 1, err, kDevErrTimeoutBase + 11);
-            if (!ok) break;
-            mbar_arrive(bars.p_ready);
+            if (!(ok = __all_sync(0xFFFFFFFFu, ok))) break;
+            mbar_arrive_warp(bars.p_ready);
           }
           if (!ok) *abort_flag = 1;
         }
@@ -703,10 +704,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = mbar_wait(bars.s_full + hb, ph & 1, err, kDevErrTimeoutBase + 10);
         // the tile's row-interval table (published by the K producer)
         if (ok) ok = mbar_wait(bars.meta_full + ms_slot, (gt / C::kMetaSlots) & 1, err, kDevErrTimeoutBase + 13);
-        if (!ok || aborted(abort_flag)) {
-          ok = false;
-          break;
-        }
+        // warp-uniform from here on (the warp arrives on barriers as one)
+        ok = __all_sync(0xFFFFFFFFu, ok && !aborted(abort_flag));
+        if (!ok) break;
         tc_fence_after();
         uint32_t r[128];   // S row: scale * log2e * r = log2e * (scale q.k + dt)
         DMA_TMEM_LD32(tS + 0, (r + 0));
@@ -716,7 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         if constexpr (C::kSepP) {
           tc_fence_before();
-          mbar_arrive(bars.s_free);   // S may be overwritten by the next Q K^T
+          mbar_arrive_warp(bars.s_free);   // S may be overwritten by the next Q K^T
         }
         if (!((j + 1) * kKeyTile <= n_full || !row_valid)) {
           // key tile not kept by every row: drop keys outside this row's interval
@@ -775,7 +775,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 64; ++c) pk[c] = p_pair(2 * c);
           if (j > 0) {
-            ok = mbar_wait(bars.o_done, (gt - 1) & 1, err, kDevErrTimeoutBase + 11);
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(bars.o_done, (gt - 1) & 1, err, kDevErrTimeoutBase + 11));
             if (!ok) break;
             tc_fence_after();
           }
@@ -794,7 +794,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // consume every o_done phase in order (PV of the previous tile), so
           // the parity of the epilogue's wait is never ambiguous
           if (j > 0) {
-            ok = mbar_wait(bars.o_done + h, (ph - 1) & 1, err, kDevErrTimeoutBase + 11);
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(bars.o_done + h, (ph - 1) & 1, err, kDevErrTimeoutBase + 11));
             if (!ok) {
               tmem_wait_st();
               break;
@@ -823,11 +823,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bars.p_ready + hb);
+        mbar_arrive_warp(bars.p_ready + hb);
       }
       // epilogue: O / l once PV of the item's last key tile is done
       if (ok) ok = mbar_wait(bars.o_done + hb, (ph0 + n_kt - 1) & 1, err, kDevErrTimeoutBase + 12);
-      if (!ok) break;
+      if (!(ok = __all_sync(0xFFFFFFFFu, ok))) break;
       tc_fence_after();
       const float inv = 1.0f / l;
       uint16_t* orow =
@@ -907,24 +907,26 @@ cudaError_t launch_d(const void* q, const void* k, const void* v, const Geometry
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::kSmemBytes);
+  cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(attn_prefill_kernel<D>), C::kSmemBytes);
   if (e != cudaSuccess) return e;
   {
-    // the warpgroups' register split must fit in what the block is launched with
-    cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, attn_prefill_kernel<D>);
-    if (e != cudaSuccess) return e;
-    if (fa.numRegs * kThreads < 128 * kRegsControl + 256 * kRegsSoftmax) return cudaErrorInvalidConfiguration;
+    // the warpgroups' register split must fit in what the block is launched
+    // with (a property of the compiled kernel: checked once)
+    static int num_regs = 0;
+    if (num_regs == 0) {
+      cudaFuncAttributes fa;
+      e = cudaFuncGetAttributes(&fa, attn_prefill_kernel<D>);
+      if (e != cudaSuccess) return e;
+      num_regs = fa.numRegs;
+    }
+    if (num_regs * kThreads < 128 * kRegsControl + 256 * kRegsSoftmax) return cudaErrorInvalidConfiguration;
   }
   const int nrep = g.Hq / g.Hkv;
   const int npairs = (nrep + 1) / 2;
   const long long n_items = static_cast<long long>(plan.n_row_tiles) * g.B * g.Hkv * npairs;
   if (n_items > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-  int dev = 0, nsm = 148;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return cudaErrorInvalidDevice;
+  const int nsm = sm_count();
+  if (nsm <= 0) return cudaErrorInvalidDevice;
   const long long nblocks = n_items < nsm ? n_items : nsm;   // persistent: one CTA per SM
   attn_prefill_kernel<D><<<static_cast<unsigned>(nblocks), kThreads, C::kSmemBytes, s>>>(
       tq, tk, tv, tk3, tv3, plan, g.B, g.Lk, g.Hq, g.Hkv, scale * kLog2e, 1.0f / scale, static_cast<uint16_t*>(out),

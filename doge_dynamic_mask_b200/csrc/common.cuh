@@ -84,6 +84,16 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t pa
   return ok != 0;
 }
 
+// One arrival per warp (barrier counts are in warps, not threads): the lanes
+// meet at a warp barrier and one lane arrives, so the barrier word takes one
+// atomic per warp instead of 32.  Callers that hand TMEM over finish and fence
+// their own tcgen05 loads / stores first (tcgen05.wait +
+// fence::before_thread_sync).
+__device__ __forceinline__ void mbar_arrive_warp(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 // Wait until the barrier's phase with the given parity has completed.  Gives
 // up after kWaitLimitCycles; then records `code` in *err and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err, uint32_t code) {

@@ -72,6 +72,40 @@ int decode_cap(int Lk, int w) {
 
 }  // namespace
 
+int sm_count() {
+  static std::mutex mu;
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == 0 && cudaDeviceGetAttribute(&cached[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    cached[dev] = 0;
+  return cached[dev];
+}
+
+cudaError_t ensure_dyn_smem(const void* func, int bytes) {
+  struct Entry {
+    const void* func;
+    int dev, bytes;
+  };
+  static std::mutex mu;
+  static Entry table[64];
+  static int n = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  int slot = -1;
+  for (int i = 0; i < n; ++i)
+    if (table[i].func == func && table[i].dev == dev) slot = i;
+  if (slot >= 0 && table[slot].bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  if (slot < 0 && n < 64) slot = n++;
+  if (slot >= 0) table[slot] = Entry{func, dev, bytes};
+  return cudaSuccess;
+}
+
 size_t prefill_plan_bytes(const Geometry& g) {
   const size_t bg = static_cast<size_t>(g.B) * g.Hkv;
   const size_t nrt = (g.Lk + kRowTile - 1) / kRowTile;

@@ -92,6 +92,11 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn get_encode_fn();
 
+// Launch-path host queries, cached per device: the SM count (0 on error), and
+// the dynamic shared-memory limit of a kernel, set once per (kernel, device).
+int sm_count();
+cudaError_t ensure_dyn_smem(const void* func, int bytes);
+
 // launchers (return cudaGetLastError() after the launch); err: device status word or nullptr
 cudaError_t launch_dt_scores(const void* v, const float* W, const float* A, int B, int L, int Hkv, int d,
                              float* dt, uint32_t* err, cudaStream_t s);

@@ -173,7 +173,7 @@ cudaError_t launch_k(const void* v, const float* W, const float* A, long long nt
   constexpr int DEPTH = 2;
   const size_t smem = static_cast<size_t>(HKV) * D / 2 * HKV * sizeof(unsigned long long);
   auto kern = dt_scores_kernel<HKV, D, K, DEPTH, WIDE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const long long warps_needed = (ntok + 32LL * K - 1) / (32LL * K);
   long long blocks = (warps_needed + kDtThreads / 32 - 1) / (kDtThreads / 32);
@@ -187,9 +187,8 @@ template <int HKV, int D>
 cudaError_t launch_t(const void* v, const float* W, const float* A, int B, int L, float* dt, cudaStream_t s) {
   constexpr int KBIG = HKV >= 8 ? 2 : 4;
   const long long ntok = static_cast<long long>(B) * L;
-  int dev = 0, nsm = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int nsm = sm_count();
+  if (nsm <= 0) return cudaErrorInvalidDevice;
   const bool wide = (reinterpret_cast<uintptr_t>(v) & 31u) == 0;
   // short inputs: one token per lane so that every SM gets warps
   if (ntok < 32LL * KBIG * 8 * 2 * nsm)
@@ -275,7 +274,7 @@ __global__ void __launch_bounds__(kDtTcThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(acc_full + b, 1);
-      mbar_init(acc_empty + b, kDtTile);
+      mbar_init(acc_empty + b, 4);   // one arrival per epilogue warp
     }
     mbar_init(fin, 1);
     *abort_flag = 0;
@@ -362,7 +361,8 @@ __global__ void __launch_bounds__(kDtTcThreads, 1)
     int it = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
       const int buf = it & 1;
-      if (!mbar_wait(acc_full + buf, (it >> 1) & 1, err, kDevErrTimeoutBase + 25) || aborted_flag(abort_flag)) {
+      const bool ok = mbar_wait(acc_full + buf, (it >> 1) & 1, err, kDevErrTimeoutBase + 25) && !aborted_flag(abort_flag);
+      if (!__all_sync(0xFFFFFFFFu, ok)) {
         *abort_flag = 1;
         break;
       }
@@ -379,7 +379,7 @@ __global__ void __launch_bounds__(kDtTcThreads, 1)
       }
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(acc_empty + buf);
+      mbar_arrive_warp(acc_empty + buf);
       const long long tok = static_cast<long long>(t) * kDtTile + row;
       if (tok < ntok) {
         const long long b = tok / L;
@@ -413,13 +413,10 @@ cudaError_t launch_tc(const void* v, const float* W, const float* A, long long n
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(dt_tc_kernel<HKV, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       T::kSmemBytes);
+  cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(dt_tc_kernel<HKV, D>), T::kSmemBytes);
   if (e != cudaSuccess) return e;
-  int dev = 0, nsm = 148;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return cudaErrorInvalidDevice;
+  const int nsm = sm_count();
+  if (nsm <= 0) return cudaErrorInvalidDevice;
   const long long n_tiles = (ntok + kDtTile - 1) / kDtTile;
   const int grid = static_cast<int>(n_tiles < nsm ? n_tiles : nsm);
   dt_tc_kernel<HKV, D><<<grid, kDtTcThreads, T::kSmemBytes, s>>>(tm, W, A, static_cast<int>(ntok), L, dt, err);

@@ -389,17 +389,14 @@ cudaError_t launch_select_prefill(const float* dt, const int32_t* lengths, const
   const int L = g.Lk;
   const int ucap = L > g.w ? g.w + kRowTile : 0;
   const size_t smem = select_smem_bytes(2 * ucap);
-  cudaError_t e = cudaFuncSetAttribute(select_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(select_prefill_kernel), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   // row tiles per CTA: runs amortise the full selection, but the grid should
   // still hold about four CTAs per SM (measured on the sparse and long
   // workloads: 2 and 4 tiles per CTA); rows of 8 tiles or more use runs of at
   // least 2
-  int dev = 0, nsm = 148;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return cudaErrorInvalidDevice;
+  const int nsm = sm_count();
+  if (nsm <= 0) return cudaErrorInvalidDevice;
   const long long tiles = static_cast<long long>(plan.n_row_tiles) * g.Hkv * g.B;
   long long tpc = (tiles + 4LL * nsm - 1) / (4LL * nsm);
   if (plan.n_row_tiles >= 8 && tpc < 2) tpc = 2;
@@ -413,8 +410,7 @@ cudaError_t launch_select_prefill(const float* dt, const int32_t* lengths, const
 cudaError_t launch_select_decode(const float* dt, const int32_t* lengths, const Geometry& g,
                                  const DecodePlan& plan, uint32_t* err, cudaStream_t s) {
   const size_t smem = select_smem_bytes(0);
-  cudaError_t e = cudaFuncSetAttribute(select_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(select_decode_kernel), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(g.Hkv, g.B);
   select_decode_kernel<<<grid, kSelThreads, smem, s>>>(dt, lengths, g.Hkv, g.Lk, g.w, plan, err);

@@ -9,10 +9,13 @@
 // shared by the Hq/Hkv query heads of the group: pure HBM traffic with ~2 FLOP
 // per byte, so the kernel is a bandwidth kernel on CUDA cores.  Split-K: one
 // CTA per (batch, kv head, 128-key chunk of the kept list); each lane owns 8
-// head dims (one 16-byte load per row), d/8 lanes cover a row, and every warp
-// issues all of its K and V row loads before using any of them.  Each CTA
-// writes an unnormalised partial (o, running max m in log2 units, sum l); a
-// second kernel merges the splits of each query head.
+// head dims (one 16-byte piece per row) and d/8 lanes cover a row.  The rows
+// travel by cp.async into shared memory, K in one group and V in a second:
+// all of a lane's row copies are in flight at once without holding
+// registers, and the scores are computed while the V rows are still
+// arriving.  Every lane reads back only the pieces it copied itself.  Each
+// CTA writes an unnormalised partial (o, running max m in log2 units, sum l);
+// a second kernel merges the splits of each query head.
 #include "common.cuh"
 
 namespace dma {
@@ -22,6 +25,17 @@ constexpr int kDecThreads = 256;
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kKeysPerWarp = kDecodeChunk / kDecWarps;   // 16
 constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// dynamic shared memory of one decode CTA: the chunk's K and V rows
+template <int D>
+constexpr int dec_smem_bytes() { return 2 * kDecodeChunk * D * 2; }
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&x)[8]) {
   x[0] = __uint_as_float(u.x << 16);
@@ -45,6 +59,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const uint16_t
   __shared__ float s_p[NREP][kDecodeChunk];
   __shared__ float s_red[kDecWarps][NREP][D];
   __shared__ float s_m[NREP], s_l[NREP];
+  extern __shared__ uint4 dyn[];
+  uint16_t* sK = reinterpret_cast<uint16_t*>(dyn);   // [kDecodeChunk][D]
+  uint16_t* sV = sK + kDecodeChunk * D;
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int Hq = Hkv * NREP;
@@ -65,26 +82,30 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const uint16_t
     bf16x8_to_f32(u, qf[r]);
   }
 
-  // issue every K and V row load of this warp first
-  uint4 kr[STEPS], vr[STEPS];
+  // issue every K row copy of this lane, then every V row copy
   int key_local[STEPS];
+  size_t rows[STEPS];
 #pragma unroll
   for (int s = 0; s < STEPS; ++s) {
     key_local[s] = warp * kKeysPerWarp + s * KPS + kg;
     // entries past the list's count are never read (key 0 stands in), so the
     // kernel does not depend on what the rest of the list buffer holds
     const int j = c0 + key_local[s] < count ? idx[key_local[s]] : 0;
-    const size_t row = ((static_cast<size_t>(b) * Lk + j) * Hkv + g) * D + dl;
-    kr[s] = __ldg(reinterpret_cast<const uint4*>(kc + row));
-    vr[s] = __ldg(reinterpret_cast<const uint4*>(vc + row));
+    rows[s] = ((static_cast<size_t>(b) * Lk + j) * Hkv + g) * D + dl;
+    cp_async16(sK + key_local[s] * D + dl, kc + rows[s]);
   }
+  cp_async_commit();
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s) cp_async16(sV + key_local[s] * D + dl, vc + rows[s]);
+  cp_async_commit();
+  cp_async_wait<1>();   // this lane's K pieces have landed
 
   // scores (log2 units)
   const float sl = scale * kLog2e;
 #pragma unroll
   for (int s = 0; s < STEPS; ++s) {
     float kf[8];
-    bf16x8_to_f32(kr[s], kf);
+    bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK + key_local[s] * D + dl), kf);
     const bool valid = c0 + key_local[s] < count;
     const float bl = bias[key_local[s]] * kLog2e;
 #pragma unroll
@@ -121,6 +142,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const uint16_t
   __syncthreads();
 
   // P V
+  cp_async_wait<0>();   // this lane's V pieces have landed
   float acc[NREP][8];
 #pragma unroll
   for (int r = 0; r < NREP; ++r)
@@ -129,7 +151,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const uint16_t
 #pragma unroll
   for (int s = 0; s < STEPS; ++s) {
     float vf[8];
-    bf16x8_to_f32(vr[s], vf);
+    bf16x8_to_f32(*reinterpret_cast<const uint4*>(sV + key_local[s] * D + dl), vf);
 #pragma unroll
     for (int r = 0; r < NREP; ++r) {
       const float p = s_p[r][key_local[s]];
@@ -187,12 +209,15 @@ __global__ void decode_combine_kernel(DecodePlan plan, int Hq, uint16_t* __restr
 template <int D, int NREP>
 cudaError_t launch_dec(const void* q, const void* k, const void* v, const Geometry& g, float scale,
                        const DecodePlan& plan, void* out, cudaStream_t s) {
+  constexpr int smem = dec_smem_bytes<D>();
+  cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(decode_attn_kernel<D, NREP>), smem);
+  if (e != cudaSuccess) return e;
   dim3 grid(plan.n_split, g.Hkv, g.B);
-  decode_attn_kernel<D, NREP><<<grid, kDecThreads, 0, s>>>(static_cast<const uint16_t*>(q),
+  decode_attn_kernel<D, NREP><<<grid, kDecThreads, smem, s>>>(static_cast<const uint16_t*>(q),
                                                            static_cast<const uint16_t*>(k),
                                                            static_cast<const uint16_t*>(v), g.Lk, g.Hkv, scale,
                                                            plan);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_combine_kernel<D><<<g.B * g.Hq, D, 0, s>>>(plan, g.Hq, static_cast<uint16_t*>(out));
   return cudaGetLastError();

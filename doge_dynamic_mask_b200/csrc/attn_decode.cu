@@ -63,6 +63,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const uint16_t
   uint16_t* sK = reinterpret_cast<uint16_t*>(dyn);   // [kDecodeChunk][D]
   uint16_t* sV = sK + kDecodeChunk * D;
 
+  pdl_wait();      // the kept lists come from the previous kernel
+  pdl_trigger();   // the combine may be scheduled
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int Hq = Hkv * NREP;
   const size_t bg = static_cast<size_t>(b) * Hkv + g;
@@ -189,6 +191,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const uint16_t
 
 template <int D>
 __global__ void decode_combine_kernel(DecodePlan plan, int Hq, uint16_t* __restrict__ out) {
+  pdl_wait();      // the partials come from the previous kernel
   const int bh = blockIdx.x;
   const float* part = plan.part + static_cast<size_t>(bh) * plan.n_split * (D + 2);
   float M = -INFINITY;
@@ -213,14 +216,11 @@ cudaError_t launch_dec(const void* q, const void* k, const void* v, const Geomet
   cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(decode_attn_kernel<D, NREP>), smem);
   if (e != cudaSuccess) return e;
   dim3 grid(plan.n_split, g.Hkv, g.B);
-  decode_attn_kernel<D, NREP><<<grid, kDecThreads, smem, s>>>(static_cast<const uint16_t*>(q),
-                                                           static_cast<const uint16_t*>(k),
-                                                           static_cast<const uint16_t*>(v), g.Lk, g.Hkv, scale,
-                                                           plan);
-  e = cudaGetLastError();
+  e = launch_after(decode_attn_kernel<D, NREP>, grid, dim3(kDecThreads), smem, s, static_cast<const uint16_t*>(q),
+                   static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v), g.Lk, g.Hkv, scale, plan);
   if (e != cudaSuccess) return e;
-  decode_combine_kernel<D><<<g.B * g.Hq, D, 0, s>>>(plan, g.Hq, static_cast<uint16_t*>(out));
-  return cudaGetLastError();
+  return launch_after(decode_combine_kernel<D>, dim3(g.B * g.Hq), dim3(D), 0, s, plan, g.Hq,
+                      static_cast<uint16_t*>(out));
 }
 
 }  // namespace

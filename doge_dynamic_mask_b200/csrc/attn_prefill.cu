@@ -336,6 +336,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // everything above overlaps the previous kernel's tail; dt, the lists and
+  // their counts come from it
+  pdl_wait();
 
   // work item i of this CTA: false when there is none left
   struct ItemInfo {
@@ -928,10 +931,9 @@ cudaError_t launch_d(const void* q, const void* k, const void* v, const Geometry
   const int nsm = sm_count();
   if (nsm <= 0) return cudaErrorInvalidDevice;
   const long long nblocks = n_items < nsm ? n_items : nsm;   // persistent: one CTA per SM
-  attn_prefill_kernel<D><<<static_cast<unsigned>(nblocks), kThreads, C::kSmemBytes, s>>>(
-      tq, tk, tv, tk3, tv3, plan, g.B, g.Lk, g.Hq, g.Hkv, scale * kLog2e, 1.0f / scale, static_cast<uint16_t*>(out),
-      err);
-  return cudaGetLastError();
+  return launch_after(attn_prefill_kernel<D>, dim3(static_cast<unsigned>(nblocks)), dim3(kThreads), C::kSmemBytes, s,
+                      tq, tk, tv, tk3, tv3, plan, g.B, g.Lk, g.Hq, g.Hkv, scale * kLog2e, 1.0f / scale,
+                      static_cast<uint16_t*>(out), err);
 }
 
 }  // namespace

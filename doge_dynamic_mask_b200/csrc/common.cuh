@@ -94,6 +94,15 @@ __device__ __forceinline__ void mbar_arrive_warp(uint64_t* bar) {
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
+// Programmatic dependent launch.  A kernel launched right after another in the
+// same stream with programmatic stream serialization (launch_after) may become
+// resident before its predecessor has finished: it runs its prologue, then
+// waits in pdl_wait() until every predecessor has completed and its memory is
+// visible.  A predecessor calls pdl_trigger() so that its dependents can be
+// scheduled before it exits.  Both are no-ops for an ordinary launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Wait until the barrier's phase with the given parity has completed.  Gives
 // up after kWaitLimitCycles; then records `code` in *err and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err, uint32_t code) {

@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(kUpdThreads) decode_update_kernel(const uint16
   __shared__ uint64_t red_key[33];
   __shared__ int red_pos[33];
   __shared__ float red_x[kUpdThreads / 32];
+  pdl_trigger();   // the decode attention may be scheduled
   const int g = blockIdx.x, b = blockIdx.y;
   const size_t bg = static_cast<size_t>(b) * Hkv + g;
   const int C = Hkv * d;

@@ -97,6 +97,24 @@ EncodeTiledFn get_encode_fn();
 int sm_count();
 cudaError_t ensure_dyn_smem(const void* func, int bytes);
 
+// Launches kern(args...) with programmatic stream serialization: it may start
+// while the stream's previous kernel finishes, and calls pdl_wait() before it
+// reads anything that kernel writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_after(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // launchers (return cudaGetLastError() after the launch); err: device status word or nullptr
 cudaError_t launch_dt_scores(const void* v, const float* W, const float* A, int B, int L, int Hkv, int d,
                              float* dt, uint32_t* err, cudaStream_t s);

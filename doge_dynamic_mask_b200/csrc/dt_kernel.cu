@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(kDtThreads) dt_scores_kernel(const uint4* __re
   constexpr int NCH = C / 16;         // 32-byte chunks per token
   static_assert(NCH % DEPTH == 0, "chunk ring must tile the row");
   extern __shared__ unsigned long long w2s[];   // [C/2][HKV] channel pairs
+  pdl_trigger();   // the next kernel (selection or attention) may be scheduled
 
   for (int i = threadIdx.x; i < (C / 2) * HKV; i += kDtThreads) {
     const int p = i / HKV, g = i % HKV;
@@ -236,6 +237,7 @@ __global__ void __launch_bounds__(kDtTcThreads, 1)
                  const float* __restrict__ A, int ntok, int L, float* __restrict__ dt, uint32_t* err) {
   using T = DtTc<HKV, D>;
   extern __shared__ unsigned char smem_raw[];
+  pdl_trigger();   // the next kernel (selection or attention) may be scheduled
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
   unsigned char* sB = smem;

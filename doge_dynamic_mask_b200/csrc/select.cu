@@ -98,6 +98,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_prefill_kernel(const fl
                                                                      uint32_t* err) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SelectSmem& sm = *reinterpret_cast<SelectSmem*>(smem_raw);
+  pdl_wait();      // dt comes from the previous kernel
+  pdl_trigger();   // the attention may be scheduled
   const int ucap = w + kRowTile;
   uint64_t* Ubuf = reinterpret_cast<uint64_t*>(smem_raw + sizeof(SelectSmem));   // two unions of ucap keys
   SelScratch sc{sm.hist, sm.cand, sm.red, sm.vars};
@@ -316,6 +318,8 @@ __global__ void __launch_bounds__(kSelThreads, 4) select_decode_kernel(const flo
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SelectSmem& sm = *reinterpret_cast<SelectSmem*>(smem_raw);
   SelScratch sc{sm.hist, sm.cand, sm.red, sm.vars};
+  pdl_wait();      // dt comes from the previous kernel
+  pdl_trigger();   // the decode attention may be scheduled
   const int g = blockIdx.x, b = blockIdx.y;
   const int len = clamp_len(lengths, b, Lk, err);
   const size_t bg = static_cast<size_t>(b) * Hkv + g;
@@ -402,9 +406,8 @@ cudaError_t launch_select_prefill(const float* dt, const int32_t* lengths, const
   if (plan.n_row_tiles >= 8 && tpc < 2) tpc = 2;
   tpc = tpc < 1 ? 1 : (tpc > kSelTilesPerCtaMax ? kSelTilesPerCtaMax : tpc);
   dim3 grid(static_cast<unsigned>((plan.n_row_tiles + tpc - 1) / tpc), g.Hkv, g.B);
-  select_prefill_kernel<<<grid, kSelThreads, smem, s>>>(dt, lengths, g.Hkv, L, g.w, static_cast<int>(tpc), plan,
-                                                        err);
-  return cudaGetLastError();
+  return launch_after(select_prefill_kernel, grid, dim3(kSelThreads), smem, s, dt, lengths, g.Hkv, L, g.w,
+                      static_cast<int>(tpc), plan, err);
 }
 
 cudaError_t launch_select_decode(const float* dt, const int32_t* lengths, const Geometry& g,
@@ -413,8 +416,8 @@ cudaError_t launch_select_decode(const float* dt, const int32_t* lengths, const 
   cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(select_decode_kernel), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(g.Hkv, g.B);
-  select_decode_kernel<<<grid, kSelThreads, smem, s>>>(dt, lengths, g.Hkv, g.Lk, g.w, plan, err);
-  return cudaGetLastError();
+  return launch_after(select_decode_kernel, grid, dim3(kSelThreads), smem, s, dt, lengths, g.Hkv, g.Lk, g.w, plan,
+                      err);
 }
 
 cudaError_t launch_prefill_bitmask(const PrefillPlan& plan, const Geometry& g, uint32_t* bitmask, cudaStream_t s) {

@@ -25,7 +25,12 @@
  *     Hkv in {1, 2, 4, 8, 16}, Hq a multiple of Hkv with Hq/Hkv <= 8,
  *     L (or Lk) in [1, 2^20], keep_window_size >= 1 (at most 8192 whenever
  *     the key length exceeds it), an sm_100 device.
- *   - Calls are asynchronous on `stream` and return a status at once; they only
+ *   - Calls are asynchronous on `stream` and ordered after the work enqueued on
+ *     it before them.  Some of a call's kernels are launched with programmatic
+ *     dependent launch: they may become resident while the previous kernel on
+ *     the stream finishes, but they wait for it to complete before reading any
+ *     input, so stream order holds for every pointer passed in.
+ *   - Calls return a status at once; they only
  *     fail synchronously on argument errors and launch errors.  Faults found
  *     on the device (a length outside [1, Lk], a bounded wait that gave up) are
  *     recorded in the workspace's status word; read them with dma_check().

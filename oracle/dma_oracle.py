@@ -23,8 +23,7 @@ Source cited throughout (the only page that defines DMA):
   [Guide §Config] section "DogeConfig 全参数详解" (num_key_value_heads, attention_bias=False,
                   keep_window_size=2048, sliding_window=None -> full causal mask).
 
-Readings taken where the pages are silent (each one is listed with its reason in
-the design notes of the repository):
+Readings taken where the pages are silent:
   * dt_proj input is the per-token value row flattened head-major
     (index h'*d + e) and projected to H_kv outputs; no bias (attention_bias=False).
   * causal and padding masking are merged into the mask BEFORE the top-k, so a
@@ -43,6 +42,8 @@ Parity status of each function (pins live in tests/test_oracle_pins.py):
                                   torch.topk on tie-free rows)
   thresholds                     pinned (rebuilds kept_mask exactly)
   attention_rows, prefill        pinned (float64 SDPA, closed forms)
+  prefill_rows                   pinned (float64 SDPA with a brute-force rank-count mask,
+                                  n_rep 1-3, padding, ties, scattered rows)
   decode_step                    pinned (float64 SDPA, closed forms)
 """
 from __future__ import annotations

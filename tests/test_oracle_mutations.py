@@ -159,3 +159,25 @@ def test_mutant_gqa_mapping_is_caught(monkeypatch):
 
     monkeypatch.setattr(oracle, "prefill", bad_prefill)
     _fails(pins.test_prefill_dense_bias_and_padding_equals_sdpa_additive_mask)
+
+
+# ---- prefill_rows mutants (the row sampler of the full-size parity tests) ----
+
+def _rows_factory(wrong_group=False, row_shift=0):
+    def rows_fn(q, k, v, dt, lengths, w, scale, b, h, rows):
+        Hq, Hkv = q.shape[2], k.shape[2]
+        g = h % Hkv if wrong_group else h // (Hq // Hkv)
+        rows = list(rows)
+        M = om.dynamic_mask_rows(dt[b, g], int(lengths[b]), q.shape[1], q.shape[1], w,
+                                 [min(max(r + row_shift, 0), q.shape[1] - 1) for r in rows])
+        return om.attention_rows(np.asarray(q[b, rows, h, :], np.float64), k[b, :, g, :], v[b, :, g, :], M, scale)
+    return rows_fn
+
+
+def test_mutant_prefill_rows_group_is_caught():
+    _fails(pins.check_prefill_rows_sdpa, _rows_factory(wrong_group=True))
+
+
+def test_mutant_prefill_rows_offset_is_caught():
+    for shift in (-1, 1):
+        _fails(pins.check_prefill_rows_sdpa, _rows_factory(row_shift=shift))

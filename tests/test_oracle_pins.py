@@ -383,3 +383,39 @@ def test_decode_equals_last_prefill_row():
     pre = oracle.prefill(q, k, v, None, None, np.array([L]), w=w, scale=0.3, dt=dt)
     dec = oracle.decode_step(q[:, L - 1], k, v, None, None, np.array([L]), w=w, scale=0.3, dt=dt)
     np.testing.assert_allclose(dec, pre[:, L - 1], rtol=1e-13, atol=1e-14)
+
+
+def check_prefill_rows_sdpa(prefill_rows, seed=15):
+    """prefill_rows (the per-(batch, query head) row sampler the full-size
+    parity tests and the CPU baseline call) against float64 SDPA with an
+    additive mask built from first principles: brute-force rank counting for
+    the kept set [Guide §DMA.3], dt on kept keys, -inf elsewhere, GQA group
+    h // n_rep [Guide §Config].  Covers n_rep 1, 2 and 3, right padding, a
+    window below the length with forced ties, and a non-contiguous row set
+    that includes the first and last rows."""
+    rng = np.random.default_rng(seed)
+    for Hq, Hkv in ((2, 2), (4, 2), (6, 2)):
+        B, L, d, w = 2, 23, 8, 5
+        q, k, v = _rand_qkv(rng, B, L, Hq, Hkv, d)
+        # few distinct dt values: many exact ties at the window boundary
+        dt = rng.choice(np.array([0.25, 0.5, 0.75, 1.5], np.float32), size=(B, Hkv, L))
+        lengths = np.array([L, 14])
+        scale = 0.31
+        add = np.full((B, Hq, L, L), -np.inf)
+        n_rep = Hq // Hkv
+        for b in range(B):
+            for h in range(Hq):
+                g = h // n_rep
+                for i in range(L):
+                    for j in brute_kept(dt[b, g], int(lengths[b]), L, L, w, i):
+                        add[b, h, i, j] = float(dt[b, g, j])
+        ref = _sdpa(q, k, v, add, scale)
+        rows = [L - 1, 0, 3, 9, 14, 13, 17]
+        for b in range(B):
+            for h in range(Hq):
+                got = prefill_rows(q, k, v, dt, lengths, w, scale, b, h, rows)
+                np.testing.assert_allclose(got, ref[b, rows, h, :], rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_rows_equals_sdpa_with_brute_force_mask():
+    check_prefill_rows_sdpa(oracle.prefill_rows)

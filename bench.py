@@ -66,6 +66,20 @@ def prefill_flops(wl, lengths):
     return 4 * wl.d * wl.Hq * kept_pairs(wl.L, wl.w, lengths)
 
 
+def kept_pairs_valid_rows(L, w, lengths):
+    """kept_pairs restricted to the valid query rows i < n of each sequence
+    (the padded rows, which the kernels also compute, left out)."""
+    total = 0
+    for n in np.asarray(lengths, dtype=np.int64):
+        vis = np.arange(1, int(n) + 1, dtype=np.int64)
+        total += int(np.minimum(vis, w).sum()) if L > w else int(vis.sum())
+    return total
+
+
+def prefill_flops_valid_rows(wl, lengths):
+    return 4 * wl.d * wl.Hq * kept_pairs_valid_rows(wl.L, wl.w, lengths)
+
+
 def decode_bytes(wl, lengths):
     """V read for dt over the whole cache + the kept K and V rows + q and out."""
     B, Lk, Hkv, d, Hq = wl.B, wl.L, wl.Hkv, wl.d, wl.Hq
@@ -91,6 +105,44 @@ def max_over_ranks(v, dist=None, device=None):
 def aggregate_throughput(units_per_rank, ms_max, world):
     """Whole-job throughput: the units every rank processed over the slowest rank's time."""
     return world * units_per_rank / (ms_max * 1e-3)
+
+
+def _free_port():
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_entry(rank, world, port, target, args):
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1",
+                      MASTER_PORT=str(port))
+    target(args)
+
+
+def spawn_ranks(world, target, args, timeout_s=1800):
+    """Runs target(args) in `world` fresh processes (spawn), one per GPU, with
+    RANK, LOCAL_RANK, WORLD_SIZE and MASTER_ADDR/PORT set as torchrun sets
+    them; returns the first non-zero exit code, or 0."""
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_entry, args=(r, world, port, target, args)) for r in range(world)]
+    for p in procs:
+        p.start()
+    rc = 0
+    t0 = time.time()
+    for p in procs:
+        p.join(timeout=max(1.0, timeout_s - (time.time() - t0)))
+        if p.exitcode is None:
+            p.kill()
+            p.join()
+            rc = rc or 1
+        else:
+            rc = rc or p.exitcode
+    return rc
 
 
 # ----------------------------------------------------------------------------
@@ -176,15 +228,6 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
-def cpu_cores():
-    try:
-        from threadpoolctl import threadpool_info
-        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
-        return int(n)
-    except Exception:
-        return os.cpu_count() or 1
-
-
 # ----------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------
@@ -250,9 +293,10 @@ def time_prefill(dma, wl, steps, warmup, flush, dev, ranks_sync):
     ms, stage = timed(dma, lambda i: step(), 0, steps, flush, ranks_sync)
     assert dma.dma_check(ws) == 0
     flops = prefill_flops(wl, lengths)
+    flops_valid = prefill_flops_valid_rows(wl, lengths)
     # dt, selector (skipped when keep_window_size >= L: no top-k) and attention
     per_step = 2 if wl.L <= wl.w else 3
-    return {"flops": flops, "ms": ms, "stage_ms": stage, "launches": per_step * steps,
+    return {"flops": flops, "flops_valid": flops_valid, "ms": ms, "stage_ms": stage, "launches": per_step * steps,
             "x": x, "ws": ws, "out": out}
 
 
@@ -364,33 +408,62 @@ def time_e2e(dma, wl, steps, warmup, dev):
     return {"tflops": prefill_flops(wl, lengths) / (ms * 1e-3) / 1e12, "ms": ms, "h2d": h2d, "d2h": d2h}
 
 
-def cpu_baseline_prefill(wl, x, budget_s=12.0):
-    """The oracle as it stands on the host cores, on a bounded sample of the
-    same workload: whole (batch, query head) slices in order, each with its
-    own dt of the whole sequence, until about budget_s seconds have passed."""
+def _oracle_worker_init():
+    from threadpoolctl import threadpool_limits
+    threadpool_limits(1)     # one BLAS thread per worker process
+
+
+def _oracle_slice(job):
+    """One (batch, query head) slice of the prefill through the oracle: dt of
+    the whole sequence, then every row of the head."""
     import oracle
+    q, k, v, W, A, lengths, w, scale, h = job
+    dt = oracle.dt_scores(v, W, A)
+    oracle.prefill_rows(q, k, v, dt, lengths, w, scale, 0, h, range(q.shape[1]))
+    return h
+
+
+class OraclePool:
+    """Worker processes for the CPU baseline: one per host core this process
+    may run on, each with one BLAS thread.  Started with spawn, so it is safe
+    to create after CUDA has been initialised."""
+
+    def __init__(self):
+        import multiprocessing as mproc
+        self.cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+        self.pool = mproc.get_context("spawn").Pool(self.cores, initializer=_oracle_worker_init)
+
+    def close(self):
+        self.pool.terminate()
+        self.pool.join()
+
+
+def cpu_baseline_prefill(wl, x, pool, budget_s=12.0):
+    """The oracle as it stands on the host cores, on a bounded sample of the
+    same workload: whole (batch, query head) slices, each with its own dt of
+    the whole sequence, spread over the pool's processes, until every slice
+    is done or about budget_s seconds have passed."""
     W = x["W"].double().cpu().numpy()
     A = x["A"].double().cpu().numpy()
-    t0 = time.perf_counter()
-    flops, done = 0, []
+    jobs = []
     for b in range(wl.B):
         q = x["q"][b:b + 1].float().cpu().numpy().astype(np.float64)
         k = x["k"][b:b + 1].float().cpu().numpy().astype(np.float64)
         v = x["v"][b:b + 1].float().cpu().numpy().astype(np.float64)
         lengths = x["lengths"][b:b + 1].cpu().numpy()
-        dt = oracle.dt_scores(v, W, A)
         for h in range(wl.Hq):
-            oracle.prefill_rows(q, k, v, dt, lengths, wl.w, wl.scale, 0, h, range(wl.L))
-            flops += prefill_flops(wl.replace(B=1, Hq=1), lengths)
-            done.append((b, h))
-            if time.perf_counter() - t0 > budget_s:
-                break
+            jobs.append(((q, k, v, W, A, lengths, wl.w, wl.scale, h), lengths))
+    t0 = time.perf_counter()
+    flops, done = 0, 0
+    for i, _ in enumerate(pool.pool.imap(_oracle_slice, [j for j, _ in jobs])):
+        flops += prefill_flops(wl.replace(B=1, Hq=1), jobs[i][1])
+        done += 1
         if time.perf_counter() - t0 > budget_s:
             break
     dt_s = time.perf_counter() - t0
-    return {"value": flops / dt_s / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-            "sample": f"{wl.name}: {len(done)} of {wl.B * wl.Hq} (batch, query head) slices, all {wl.L} rows "
-                      f"each, dt included, {dt_s:.1f} s"}
+    return {"value": flops / dt_s / 1e12, "unit": "TFLOP/s", "cores": pool.cores, "kind": "oracle",
+            "sample": f"{wl.name}: {done} of {wl.B * wl.Hq} (batch, query head) slices, all {wl.L} rows "
+                      f"each, dt included, {dt_s:.1f} s over {pool.cores} worker processes (one BLAS thread each)"}
 
 
 def run_only(args):
@@ -479,6 +552,7 @@ def run_ours(args):
             oms = rank_max(o["ms"])
             a_ms = rank_max(o["stage_ms"][2])
             others[name] = {"value": round(aggregate_throughput(o["flops"], oms, world) / 1e12, 3), "unit": "TFLOP/s",
+                            "valid_rows_value": round(aggregate_throughput(o["flops_valid"], oms, world) / 1e12, 3),
                             "ms_per_step": round(oms, 5),
                             "attention_tflops": round(o["flops"] / (a_ms * 1e-3) / 1e12, 2),
                             "attention_frac": round(o["flops"] / (a_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
@@ -515,7 +589,11 @@ def run_ours(args):
                      "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": round(e2e["ms"], 4)}
     if rank == 0:
         x = make_inputs(wl, device="cpu")
-        result["cpu_baseline"] = cpu_baseline_prefill(wl, x)
+        pool = OraclePool()
+        try:
+            result["cpu_baseline"] = cpu_baseline_prefill(wl, x, pool)
+        finally:
+            pool.close()
         print(json.dumps(result), flush=True)
     if pg is not None:
         pg.barrier()
@@ -530,10 +608,14 @@ def run_reference(args):
     x = make_inputs(wl, device="cpu")
     lengths = x["lengths"].numpy()
     per_step = []
-    for i in range(args.warmup + args.steps):
-        r = cpu_baseline_prefill(wl, x, budget_s=8.0)
-        if i >= args.warmup:
-            per_step.append(r)
+    pool = OraclePool()
+    try:
+        for i in range(args.warmup + args.steps):
+            r = cpu_baseline_prefill(wl, x, pool, budget_s=8.0)
+            if i >= args.warmup:
+                per_step.append(r)
+    finally:
+        pool.close()
     value = statistics.mean(r["value"] for r in per_step)
     total_flops = prefill_flops(wl, lengths)
     line = {"metric": METRIC, "impl": "reference", "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
@@ -566,7 +648,15 @@ def main():
         run_reference(args)
     elif args.only:
         run_only(args)
+    elif args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # not launched by torchrun: start one process per GPU here
+        if torch.cuda.device_count() < args.gpus:
+            sys.exit(f"bench.py --gpus {args.gpus}: only {torch.cuda.device_count()} GPU(s) visible")
+        sys.exit(spawn_ranks(args.gpus, run_ours, args))
     else:
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        if world != args.gpus and args.gpus != 1:
+            sys.exit(f"bench.py --gpus {args.gpus} under a launcher with WORLD_SIZE={world}")
         run_ours(args)
 
 

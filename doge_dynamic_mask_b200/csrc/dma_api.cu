@@ -22,14 +22,16 @@ cudaError_t stage_mark(int i, cudaStream_t s) {
   return cudaEventRecord(static_cast<cudaEvent_t>(g_stage_events[i]), s);
 }
 
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool hkv_ok(int Hkv) { return Hkv == 1 || Hkv == 2 || Hkv == 4 || Hkv == 8 || Hkv == 16; }
+
+}  // namespace
+
 dma_status_t cuda_fail(cudaError_t e) {
   g_last_cuda_error = static_cast<int>(e);
   return DMA_ERR_CUDA;
 }
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-bool hkv_ok(int Hkv) { return Hkv == 1 || Hkv == 2 || Hkv == 4 || Hkv == 8 || Hkv == 16; }
 
 // sm_100 check, cached per device.
 dma_status_t device_ok() {
@@ -48,6 +50,8 @@ dma_status_t device_ok() {
   }
   return cached[dev] == 1 ? DMA_OK : DMA_ERR_UNSUPPORTED;
 }
+
+namespace {
 
 // Shape checks shared by every entry point (Lk is the key axis).
 dma_status_t check_shape(int B, int Lk, int Hq, int Hkv, int d, int w) {
@@ -327,10 +331,13 @@ dma_status_t dma_forward_prefill(const void* q, const void* k, const void* v, co
   return DMA_OK;
 }
 
-dma_status_t dma_decode_step(const void* q, const void* k_cache, const void* v_cache, const float* W_dt,
-                             const float* A, const int32_t* lengths, int B, int Lk, int Hq, int Hkv, int d,
-                             int keep_window_size, float scale, const float* dt_in, void* out, void* workspace,
-                             size_t ws_bytes, dma_stream_t stream) {
+}  // extern "C"
+
+namespace dma {
+dma_status_t check_decode_args(const void* q, const void* k_cache, const void* v_cache, const float* W_dt,
+                               const float* A, const int32_t* lengths, int B, int Lk, int Hq, int Hkv, int d,
+                               int keep_window_size, float scale, const float* dt_in, const void* out,
+                               const void* workspace) {
   if (!q || !k_cache || !v_cache || !out || !workspace) return DMA_ERR_INVALID_ARG;
   if (!dt_in && (!W_dt || !A)) return DMA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned16(workspace) ||
@@ -340,7 +347,19 @@ dma_status_t dma_decode_step(const void* q, const void* k_cache, const void* v_c
   if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return DMA_ERR_INVALID_ARG;
   dma_status_t st = check_shape(B, Lk, Hq, Hkv, d, keep_window_size);
   if (st != DMA_OK) return st;
-  if ((st = device_ok()) != DMA_OK) return st;
+  return device_ok();
+}
+}  // namespace dma
+
+extern "C" {
+
+dma_status_t dma_decode_step(const void* q, const void* k_cache, const void* v_cache, const float* W_dt,
+                             const float* A, const int32_t* lengths, int B, int Lk, int Hq, int Hkv, int d,
+                             int keep_window_size, float scale, const float* dt_in, void* out, void* workspace,
+                             size_t ws_bytes, dma_stream_t stream) {
+  const dma_status_t st = check_decode_args(q, k_cache, v_cache, W_dt, A, lengths, B, Lk, Hq, Hkv, d,
+                                            keep_window_size, scale, dt_in, out, workspace);
+  if (st != DMA_OK) return st;
   const Geometry g{B, 1, Lk, Hq, Hkv, d, keep_window_size};
   if (ws_bytes < decode_plan_bytes(g)) return DMA_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

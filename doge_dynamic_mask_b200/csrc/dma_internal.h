@@ -6,6 +6,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "../../include/dma.h"
+
 namespace dma {
 
 // Query rows per prefill row tile and keys per attention key tile.
@@ -114,6 +116,17 @@ cudaError_t launch_after(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t s
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
+
+// Entry-point helpers shared by the C ABI's translation units: record a CUDA
+// error for dma_last_cuda_error() and return DMA_ERR_CUDA; the sm_100 device
+// check; and the argument checks of dma_decode_step (everything it verifies
+// before it enqueues work, workspace size aside).
+dma_status_t cuda_fail(cudaError_t e);
+dma_status_t device_ok();
+dma_status_t check_decode_args(const void* q, const void* k_cache, const void* v_cache, const float* W_dt,
+                               const float* A, const int32_t* lengths, int B, int Lk, int Hq, int Hkv, int d,
+                               int keep_window_size, float scale, const float* dt_in, const void* out,
+                               const void* workspace);
 
 // launchers (return cudaGetLastError() after the launch); err: device status word or nullptr
 cudaError_t launch_dt_scores(const void* v, const float* W, const float* A, int B, int L, int Hkv, int d,

@@ -100,7 +100,31 @@ DMA_API dma_status_t dma_dt_scores(const void* v, const float* W_dt, const float
  *                is 1 iff key j is kept.  Expanded from the compact plan the
  *                attention kernels read (debug/test use; it is Lq*Lk bits).
  *   workspace    dma_workspace_size(B, Lq, Lk, Hkv, Hkv, 64, keep_window_size) bytes
- *                or more; on return it holds the compact plan.
+ *                or more; on return it holds the compact plan (the block map the
+ *                attention kernels read), laid out as below.
+ *
+ * Compact plan layout in the workspace.  Offsets are in bytes; each array
+ * starts at the next multiple of 256 after the previous one ends; the first
+ * 256 bytes are the header (status word at offset 0).
+ *   Prefill geometry (Lq == Lk == L), n_rt = ceil(L / 128) row tiles,
+ *   tiles = B * Hkv * n_rt ordered ((b * Hkv + g) * n_rt + t),
+ *   cap = roundup(L > w ? min(w + 127, L) : L, 128):
+ *     dt     [B, Hkv, L]        float32   (written by dma_forward_prefill when dt_in is NULL)
+ *     tau    [B, Hkv, L]        uint64    row thresholds (as tau_out)
+ *     idx    [tiles, cap]       int32     the keys any row of the tile keeps: first
+ *                                         those every row keeps, then the others, each
+ *                                         class in ascending key order
+ *     bias   [tiles, cap]       float32   dt of the listed key
+ *     span   [tiles, cap]       uint32    lo | hi << 16: the tile rows [lo, hi) keeping it
+ *     counts [tiles]            int32 x2  (n_full, n_total): entries [0, n_full) are kept
+ *                                         by every row; entries from n_total up to the
+ *                                         next multiple of 128 are padding (span 0)
+ *     kbase  [tiles, cap / 128] int32     j0 when 128-entry block k lists exactly
+ *                                         j0, j0+1, ..., else -1
+ *   Decode geometry (Lq == 1), cap = roundup(min(Lk, w), 128):
+ *     dt [B, Hkv, Lk] float32, tau [B, Hkv] uint64, idx [B, Hkv, cap] int32 (kept
+ *     keys ascending), bias [B, Hkv, cap] float32, count [B, Hkv] int32, then the
+ *     split-K partials of dma_decode_step.
  */
 DMA_API dma_status_t dma_build_mask(const float* dt, const int32_t* lengths, int B, int Hkv, int Lq, int Lk,
                             int keep_window_size, uint64_t* tau_out, uint32_t* bitmask_out, void* workspace,
@@ -189,7 +213,12 @@ DMA_API dma_status_t dma_decode_step_cached(const void* q, const void* k_cache, 
  *     exceeds 64 MiB (roughly B * Hkv * Lk above 15.7 million cached keys).
  *   - The first call on a device looks up the array's device address on that
  *     device (cudaGetSymbolAddress, with the device current); make that first
- *     call before any stream capture.
+ *     call before any stream capture.  The address is cached per device and
+ *     context: after the device's context is destroyed and made anew
+ *     (cudaDeviceReset), the next call looks it up again, and that call too
+ *     belongs before any stream capture.
+ *   - Arguments are checked exactly as dma_decode_step checks them before
+ *     anything is enqueued; a rejected call enqueues nothing.
  *   - Every call on every stream shares the one array and it keeps the last
  *     call's contents; calls that overlap on the GPU race, so serialise them
  *     (one stream, or events).  The status word is cleared at the start of

@@ -65,3 +65,17 @@ def test_dense_eq_flops_and_decode_bytes():
     short = lengths.copy()
     short[0] = 100
     assert bench.decode_bytes(dec, short) == bench.decode_bytes(dec, lengths) - dec.Hkv * 2 * (dec.w - 100) * dec.d * 2
+
+
+def test_valid_rows_pairs_equal_the_oracle_mask_count_over_valid_rows():
+    rng = np.random.default_rng(22)
+    for trial in range(12):
+        L = int(rng.integers(1, 60))
+        w = int(rng.integers(1, 70))
+        lengths = rng.integers(1, L + 1, size=3).astype(np.int32)
+        dt = rng.uniform(0.01, 1.0, size=(3, 1, L)).astype(np.float32)
+        kept = oracle.kept_mask(dt, lengths, L, L, w)
+        want = sum(int(kept[b, 0, :lengths[b]].sum()) for b in range(3))
+        assert bench.kept_pairs_valid_rows(L, w, lengths) == want, (trial, L, w, lengths)
+    # full-length sequences: the valid-rows count is the whole count
+    assert bench.kept_pairs_valid_rows(2048, 2048, [2048] * 2) == bench.kept_pairs(2048, 2048, [2048] * 2)

@@ -54,3 +54,27 @@ def test_single_process_needs_no_group():
     import bench
     assert bench.max_over_ranks(3.5) == 3.5
     assert bench.aggregate_throughput(2.0, 1000.0, 1) == pytest.approx(2.0)
+
+
+def _spawned_target(args):
+    """A rank started by bench.spawn_ranks: joins a gloo group from the
+    environment the launcher set and reports what it sees."""
+    dist.init_process_group("gloo")
+    try:
+        import bench
+        rank, world = dist.get_rank(), dist.get_world_size()
+        ms = bench.max_over_ranks(20.0 + rank, dist, torch.device("cpu"))
+        with open(os.path.join(args["dir"], f"rank{rank}.txt"), "w") as f:
+            f.write(f"{rank} {world} {os.environ['LOCAL_RANK']} {ms}")
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_spawn_ranks_starts_one_process_per_rank(tmp_path):
+    """The launch path bench.py takes for --gpus N outside torchrun."""
+    import bench
+    rc = bench.spawn_ranks(2, _spawned_target, {"dir": str(tmp_path)}, timeout_s=180)
+    assert rc == 0
+    got = sorted(open(tmp_path / f"rank{r}.txt").read().split() for r in range(2))
+    assert got == [["0", "2", "0", "21.0"], ["1", "2", "1", "21.0"]]

@@ -6,7 +6,8 @@ and forbids raw cudaMalloc, or plain C callers without a device allocator): it
 keeps its scratch in a fixed array inside the library.  Its output must match
 the ordinary dma_decode_step (which takes a caller-provided workspace) within
 the output tolerance used by every parity test here, on two calls in a row
-(the second call reuses the array the first one left behind).
+(the second call reuses the array the first one left behind), and so must
+the float64 oracle's; a second call must not change the device's free memory.
 
 This file is named so that pytest collects it last.
 """
@@ -55,6 +56,32 @@ def test_noalloc_decode_matches_workspace_decode_twice(dma):
         err = (got.float() - want.float()).abs().cpu().numpy()
         assert np.isfinite(err).all()
         assert err.max() <= OUT_MAX and err.mean() <= OUT_MEAN, (seed, err.max(), err.mean())
+
+
+def test_noalloc_decode_matches_oracle_and_allocates_nothing(dma):
+    """Against the float64 oracle directly, on two calls in a row; the second
+    call (after the first has loaded the kernels) leaves the device's free
+    memory exactly as it was."""
+    import oracle
+    lib = dma.raw()
+    wl = Workload("noalloc", "decode", B=2, L=5000, Hq=8, Hkv=4, d=128, w=1024, a_lo=-2.0, a_hi=-0.1,
+                  seed=303, len_lo=900, len_hi=5000)
+    xh = make_inputs(wl)
+    x = {k: v.cuda() for k, v in xh.items()}
+    f64 = lambda t: t.float().numpy().astype(np.float64)
+    want = oracle.decode_step(f64(xh["q"]), f64(xh["k"]), f64(xh["v"]), xh["W"].double().numpy(),
+                              xh["A"].double().numpy(), xh["lengths"].numpy(), wl.w, wl.scale)
+    outs = [torch.full_like(x["q"], float("nan")) for _ in range(2)]
+    assert _noalloc(lib, x, wl, outs[0]) == 0
+    torch.cuda.synchronize()
+    free_before = torch.cuda.mem_get_info()[0]
+    assert _noalloc(lib, x, wl, outs[1]) == 0
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free_before
+    for out in outs:
+        err = np.abs(out.float().cpu().numpy() - want)
+        assert np.isfinite(err).all()
+        assert err.max() <= OUT_MAX and err.mean() <= OUT_MEAN, (err.max(), err.mean())
 
 
 def test_noalloc_rejects_steps_beyond_its_scratch(dma):

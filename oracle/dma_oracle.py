@@ -45,6 +45,12 @@ Parity status of each function (pins live in tests/test_oracle_pins.py):
   prefill_rows                   pinned (float64 SDPA with a brute-force rank-count mask,
                                   n_rep 1-3, padding, ties, scattered rows)
   decode_step                    pinned (float64 SDPA, closed forms)
+  rms_norm                       pinned (hand example, unit mean square, scale invariance)
+  rope_angles, rope              pinned (2-D closed form, complex-number form, relative
+                                  position, composition, identity at position 0)
+  prologue                       pinned (pair lengths show norm-then-rotate, position 0 is
+                                  the plain norm, relative-position invariance under a
+                                  shifted offset, untouched cache rows, V appended as is)
 """
 from __future__ import annotations
 
@@ -266,3 +272,74 @@ def decode_step(q, k_cache, v_cache, W, A, lengths, w, scale, dt=None, batches=N
                 out[ob, h, :] = attention_rows(np.asarray(q[b, h][None, :], dtype=np.float64),
                                                kb[:, g, :], vb[:, g, :], M, scale)[0]
     return out
+
+
+# --------------------------------------------------------------------------
+# Prologue: q_norm / k_norm, rotary position embedding, KV-cache append
+#   [Guide §DMA.1-2]  section "动态掩码注意力（DMA）", forward-chain steps 1 and 2:
+#                     after q_proj/k_proj/v_proj, Q and K each pass an RMSNorm
+#                     over head_dim (q_norm / k_norm), then the rotary position
+#                     embedding (apply_rotary_pos_emb); with a cache, K and V
+#                     are appended to it (past_key_values.update).
+#   [Guide §Modules]  section "从源码理解两大核心模块": RMSNorm and RoPE are the
+#                     Llama implementations; [Guide §Residual] DogeRMSNorm is the
+#                     T5-style norm (learnable elementwise scale, variance in fp32).
+#   [Guide §Config]   rms_norm_eps = 1e-6; rope_parameters (rope_theta) has no
+#                     default on the page.
+# Readings taken where the pages are silent:
+#   * RMSNorm: y = w * x / sqrt(mean(x^2) + eps) over the d channels of one head.
+#   * RoPE (the Llama convention): channel i < d/2 pairs with channel i + d/2;
+#     the pair is rotated by the angle pos * theta^(-2i/d):
+#       (a, b) -> (a cos - b sin, b cos + a sin).
+#   * token t of sequence b sits at position positions[b] + t, and is written to
+#     the cache row of that position.
+#   * norm first, then rotation (the order of step 1); V is appended unchanged.
+# --------------------------------------------------------------------------
+
+def rms_norm(x, w, eps):
+    """RMSNorm over the last axis, float64: w * x / sqrt(mean(x^2) + eps)."""
+    x = np.asarray(x, dtype=np.float64)
+    ms = (x * x).mean(axis=-1, keepdims=True)
+    return np.asarray(w, dtype=np.float64) * (x / np.sqrt(ms + eps))
+
+
+def rope_angles(pos, d, theta):
+    """Rotation angles [len(pos), d/2]: pos * theta^(-2i/d), float64."""
+    i = np.arange(d // 2, dtype=np.float64)
+    inv_freq = np.power(float(theta), -2.0 * i / d)
+    return np.asarray(pos, dtype=np.float64)[:, None] * inv_freq[None, :]
+
+
+def rope(x, pos, theta):
+    """Rotary embedding of x [..., n, H, d] at positions pos [n] (Llama pairing)."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    ang = rope_angles(pos, d, theta)                   # [n, d/2]
+    c = np.cos(ang)[:, None, :]
+    s = np.sin(ang)[:, None, :]
+    a, b = x[..., : d // 2], x[..., d // 2:]
+    return np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
+
+
+def prologue(q, k, v, q_norm_w, k_norm_w, eps, theta, positions, k_cache, v_cache):
+    """Steps 1-2 of the attention forward for new tokens.
+
+    q [B, L, H_q, d], k / v [B, L, H_kv, d] projected states; q_norm_w / k_norm_w [d];
+    positions [B] cache offset of each sequence's first new token;
+    k_cache / v_cache [B, Lmax, H_kv, d] (not modified).
+    Returns (q_out [B, L, H_q, d], k_cache_out, v_cache_out) in float64, the
+    caches with rows positions[b] .. positions[b] + L - 1 replaced.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, L = q.shape[:2]
+    kc = np.array(k_cache, dtype=np.float64, copy=True)
+    vc = np.array(v_cache, dtype=np.float64, copy=True)
+    q_out = np.empty_like(q)
+    for b in range(B):
+        pos = int(positions[b]) + np.arange(L)
+        q_out[b] = rope(rms_norm(q[b], q_norm_w, eps), pos, theta)
+        kc[b, pos] = rope(rms_norm(k[b], k_norm_w, eps), pos, theta)
+        vc[b, pos] = v[b]
+    return q_out, kc, vc

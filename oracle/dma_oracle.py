@@ -51,6 +51,11 @@ Parity status of each function (pins live in tests/test_oracle_pins.py):
   prologue                       pinned (pair lengths show norm-then-rotate, position 0 is
                                   the plain norm, relative-position invariance under a
                                   shifted offset, untouched cache rows, V appended as is)
+  cdmoe_logits                   pinned (float64 matmul against explicit index loops)
+  cdmoe_route                    pinned (brute force over all K*K experts on tie-free logits,
+                                  closed form on constant logits, torch.topk per domain)
+  cdmoe_experts, cdmoe           pinned (one expert = silu(h.d) u, equal scores = plain mean,
+                                  linearity in up_embed, a hand-worked two-expert example)
 """
 from __future__ import annotations
 
@@ -343,3 +348,82 @@ def prologue(q, k, v, q_norm_w, k_norm_w, eps, theta, positions, k_cache, v_cach
         kc[b, pos] = rope(rms_norm(k[b], k_norm_w, eps), pos, theta)
         vc[b, pos] = v[b]
     return q_out, kc, vc
+
+
+# --------------------------------------------------------------------------
+# CDMoE routing   [Guide §CDMoE]  section "跨域 MoE（CDMoE）：在稠密 checkpoint 上“叠加”稀疏专家"
+#   router_gate maps the hidden state to num_keys * 2 logits; a top-k runs on
+#   each of the two domains x and y (num_keys = floor(sqrt(num_experts)));
+#   their Cartesian product gives the expert indices; the experts are rows of
+#   two embedding tables (down_embed, up_embed [num_experts, hidden_size]):
+#   looked up and applied to the hidden state as down-projection -> activation
+#   -> up-projection, added to the shared expert's output.
+#   [Guide §Config]  num_experts = 16384, num_experts_per_tok = 64 (the top-k),
+#   hidden_act = "silu", mlp_bias = False, norm_topk_prob = False.
+# Readings taken where the pages are silent:
+#   * logits [T, 2K]: columns [0, K) are domain x, [K, 2K) domain y; no bias.
+#   * each domain keeps its k = num_experts_per_tok best keys (ties: lower key
+#     index); the product pair (a, b) scores s_x[a] + s_y[b] (float32 sum, the
+#     precision the logits are handed on in) and names expert a * K + b; the
+#     token keeps the k best of the k * k pairs (ties: lower expert index).
+#   * routing weights: softmax over the k kept scores (norm_topk_prob = False
+#     adds no further scaling).
+#   * expert e contributes weight_e * silu(h . down_embed[e]) * up_embed[e].
+# --------------------------------------------------------------------------
+
+def cdmoe_logits(h, W_router):
+    """router_gate: h [T, hidden] @ W_router [hidden, 2K], float64."""
+    return np.asarray(h, dtype=np.float64) @ np.asarray(W_router, dtype=np.float64)
+
+
+def _topk_stable(vals, k):
+    """Indices of the k largest values, larger first, ties to the lower index."""
+    order = np.argsort(-np.asarray(vals, dtype=np.float64), kind="stable")
+    return order[:k]
+
+
+def cdmoe_route(logits, k):
+    """Expert indices [T, k] (int64) and scores [T, k] (float32) from float32
+    router logits [T, 2K]: top-k per domain, then the k best of their product."""
+    logits = np.asarray(logits, dtype=np.float32)
+    T, twoK = logits.shape
+    K = twoK // 2
+    experts = np.empty((T, k), dtype=np.int64)
+    scores = np.empty((T, k), dtype=np.float32)
+    for t in range(T):
+        lx, ly = logits[t, :K], logits[t, K:]
+        ix = _topk_stable(lx, k)
+        iy = _topk_stable(ly, k)
+        cand_s = (lx[ix][:, None] + ly[iy][None, :]).astype(np.float32).ravel()   # float32 sums
+        cand_e = (ix[:, None] * K + iy[None, :]).ravel()
+        # best score first; equal scores: lower expert index first
+        order = np.lexsort((cand_e, -cand_s.astype(np.float64)))[:k]
+        experts[t] = cand_e[order]
+        scores[t] = cand_s[order]
+    return experts, scores
+
+
+def cdmoe_experts(h, experts, scores, down_embed, up_embed):
+    """Routed output [T, hidden], float64: sum over the kept experts of
+    softmax(scores)_e * silu(h . down_embed[e]) * up_embed[e]."""
+    h = np.asarray(h, dtype=np.float64)
+    D = np.asarray(down_embed, dtype=np.float64)
+    U = np.asarray(up_embed, dtype=np.float64)
+    out = np.empty_like(h)
+    for t in range(h.shape[0]):
+        s = np.asarray(scores[t], dtype=np.float64)
+        wts = np.exp(s - s.max())
+        wts = wts / wts.sum()
+        a = D[experts[t]] @ h[t]                  # down-projection: one scalar per expert
+        act = a / (1.0 + np.exp(-a))              # silu
+        out[t] = (wts * act) @ U[experts[t]]      # up-projection
+    return out
+
+
+def cdmoe(h, W_router, down_embed, up_embed, k, logits=None):
+    """Routed CDMoE output [T, hidden] (float64), experts [T, k], scores [T, k].
+    logits, when given, are the float32 router logits [T, 2K] to route on."""
+    if logits is None:
+        logits = cdmoe_logits(h, W_router).astype(np.float32)
+    experts, scores = cdmoe_route(logits, k)
+    return cdmoe_experts(h, experts, scores, down_embed, up_embed), experts, scores

@@ -54,6 +54,8 @@ Parity status of each function (pins live in tests/test_oracle_pins.py):
   cdmoe_logits                   pinned (float64 matmul against explicit index loops)
   cdmoe_route                    pinned (brute force over all K*K experts on tie-free logits,
                                   closed form on constant logits, torch.topk per domain)
+  prefill_backward               pinned (float64 torch.autograd of an independent forward,
+                                  central finite differences, planted mistakes)
   cdmoe_experts, cdmoe           pinned (one expert = silu(h.d) u, equal scores = plain mean,
                                   linearity in up_embed, a hand-worked two-expert example)
 """
@@ -427,3 +429,77 @@ def cdmoe(h, W_router, down_embed, up_embed, k, logits=None):
         logits = cdmoe_logits(h, W_router).astype(np.float32)
     experts, scores = cdmoe_route(logits, k)
     return cdmoe_experts(h, experts, scores, down_embed, up_embed), experts, scores
+
+
+# --------------------------------------------------------------------------
+# Backward of the prefill path, the kept-key selection held fixed
+#   [Guide §DMA.3] the closing paragraph: dt comes from the cached value
+#   states, so the training stage learns end to end which history tokens to
+#   mask; [Guide] the architecture list's item 1 (training uses self-attention
+#   tied to the value states).
+# Readings taken where the pages are silent:
+#   * the top-k is a selection, not a function with a gradient: the kept set
+#     of every row is held fixed, and gradients flow through the dt values of
+#     the kept keys (masked entries are constants);
+#   * the float32 rounding of dt for the mask passes gradients unchanged.
+# For L = sum(out * dout):
+#   dP = dO V^T, D_i = dO_i . O_i, dS = P (dP - D), dQ = scale dS K,
+#   dK = scale dS^T Q, dV = P^T dO (+ the dt path below),
+#   d_dt[g, j] = sum over the group's heads and rows of dS[., j];
+#   dt = exp(A softplus(x)):  dA = sum d_dt dt softplus(x),
+#   dx = d_dt dt A sigmoid(x),  dW = v_flat^T dx,  dV_flat += dx W^T.
+# --------------------------------------------------------------------------
+
+def prefill_backward(q, k, v, W, A, lengths, w, scale, dout, dt_fixed=None):
+    """Gradients of sum(prefill(...) * dout), float64.
+
+    Returns dq [B,L,Hq,d], dk [B,L,Hkv,d], dv [B,L,Hkv,d] (attention and dt
+    paths), d_dt [B,Hkv,L], dW [Hkv*d, Hkv], dA [Hkv].  dt_fixed, when given,
+    is the float32 dt the mask is built from (the kernels' own dt): the
+    selection and bias use it, while the dt chain still starts from W and A.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    A = np.asarray(A, dtype=np.float64)
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    n_rep = Hq // Hkv
+    # forward quantities of the dt chain  [Guide §DMA.3]
+    x = v.reshape(B, L, Hkv * d) @ W                       # [B, L, Hkv]
+    sp = softplus(x)
+    dt64 = np.exp(A[None, None, :] * sp)                   # [B, L, Hkv]
+    dt32 = dt64.transpose(0, 2, 1).astype(np.float32) if dt_fixed is None else np.asarray(dt_fixed, np.float32)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    d_dt = np.zeros((B, Hkv, L))
+    for b in range(B):
+        for g in range(Hkv):
+            M = dynamic_mask_rows(dt32[b, g], int(lengths[b]), L, L, w, range(L))    # [L, L]
+            Kg, Vg = k[b, :, g, :], v[b, :, g, :]
+            for r in range(n_rep):
+                h = g * n_rep + r
+                Q, dO = q[b, :, h, :], dout[b, :, h, :]
+                s = scale * (Q @ Kg.T) + M
+                s = s - s.max(axis=1, keepdims=True)
+                P = np.exp(s)
+                P = P / P.sum(axis=1, keepdims=True)
+                O = P @ Vg
+                dP = dO @ Vg.T
+                Dr = (dO * O).sum(axis=1, keepdims=True)
+                dS = P * (dP - Dr)
+                dq[b, :, h, :] = scale * (dS @ Kg)
+                dk[b, :, g, :] += scale * (dS.T @ Q)
+                dv[b, :, g, :] += P.T @ dO
+                d_dt[b, g, :] += dS.sum(axis=0)
+    ddt = d_dt.transpose(0, 2, 1)                          # [B, L, Hkv]
+    dA = (ddt * dt64 * sp).sum(axis=(0, 1))
+    sig = 1.0 / (1.0 + np.exp(-x))
+    dx = ddt * dt64 * A[None, None, :] * sig               # [B, L, Hkv]
+    v_flat = v.reshape(B * L, Hkv * d)
+    dW = v_flat.T @ dx.reshape(B * L, Hkv)
+    dv += (dx.reshape(B * L, Hkv) @ W.T).reshape(B, L, Hkv, d)
+    return dq, dk, dv, d_dt, dW, dA

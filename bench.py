@@ -350,6 +350,99 @@ def time_decode_cached(dma, wl, steps, warmup, flush, dev, ranks_sync):
     return {"bytes": nbytes, "ms": ms, "stage_ms": stage, "launches": 3 * steps}
 
 
+def time_prologue(dma, wl, steps, warmup, flush, dev, ranks_sync):
+    """The prologue (q/k RMSNorm, rotary embedding, KV-cache append) over the
+    workload's L tokens per sequence, written at the start of an L-row cache."""
+    from doge_dynamic_mask_b200.workloads import make_prologue_inputs
+    x = make_prologue_inputs(wl.B, wl.L, wl.L, wl.Hq, wl.Hkv, wl.d, wl.seed, device=dev,
+                             positions=[0] * wl.B)
+    ws = dma.new_workspace(256, dev)
+    q_out = torch.empty_like(x["q"])
+
+    def step(i):
+        dma.dma_prologue(x["q"], x["k"], x["v"], x["q_w"], x["k_w"], x["positions"], x["k_cache"], x["v_cache"],
+                         q_out=q_out, workspace=ws)
+
+    for i in range(warmup):
+        step(i)
+        flush.zero_()
+    assert dma.dma_check(ws) == 0
+    ranks_sync()
+    ms = run_steps(dma, step, 0, steps, flush)
+    ranks_sync()
+    assert dma.dma_check(ws) == 0
+    # every projected row read once and written once (q to q_out, k and v to the cache)
+    nbytes = 2 * wl.B * wl.L * (wl.Hq + 2 * wl.Hkv) * wl.d * 2
+    del x
+    return {"bytes": nbytes, "ms": sum(ms) / len(ms), "launches": steps}
+
+
+def time_backward(dma, wl, steps, warmup, flush, dev, ranks_sync):
+    """The backward of the prefill step (selection held fixed) on the
+    workload: dt, the kept-key lists, the attention backward and the dt chain."""
+    x = make_inputs(wl, device=dev)
+    lengths = x["lengths"].cpu().numpy()
+    out = torch.empty_like(x["q"])
+    dma.dma_forward_prefill(x["q"], x["k"], x["v"], x["W"], x["A"], x["lengths"], wl.w, out=out)
+    g = torch.Generator(device=dev).manual_seed(wl.seed + 100)
+    dout = torch.randn(x["q"].shape, generator=g, device=dev).to(torch.bfloat16)
+    ws = dma.new_workspace(dma.dma_backward_workspace_size(wl.B, wl.L, wl.Hq, wl.Hkv, wl.d, wl.w), dev)
+
+    def step(i):
+        dma.dma_backward_prefill(x["q"], x["k"], x["v"], x["W"], x["A"], x["lengths"], wl.w, out, dout,
+                                 workspace=ws)
+
+    for i in range(warmup):
+        step(i)
+        flush.zero_()
+    assert dma.dma_check(ws) == 0
+    ranks_sync()
+    ms = run_steps(dma, step, 0, steps, flush)
+    ranks_sync()
+    split = run_steps(dma, step, steps, steps, flush, stages=True)
+    assert dma.dma_check(ws) == 0
+    # the five products of an attention backward (S, dP, dQ, dK, dV): 10 d FLOPs per kept pair per query head
+    flops = 10 * wl.d * wl.Hq * kept_pairs(wl.L, wl.w, lengths)
+    n = len(split)
+    del x
+    return {"flops": flops, "ms": sum(ms) / len(ms), "stage_ms": [sum(v[k] for v in split) / n for k in range(3)],
+            "launches": 5 * steps}
+
+
+CDMOE = {"T": 8192, "hidden": 1024, "num_experts": 16384, "top_k": 64, "seed": 11}
+
+
+def time_cdmoe(dma, steps, warmup, flush, dev, ranks_sync):
+    """CDMoE routing at DogeConfig's defaults (hidden 1024, 16384 experts, 64
+    per token) for 8192 tokens: router GEMM, routing, embedding-table experts."""
+    from doge_dynamic_mask_b200.workloads import make_cdmoe_inputs
+    c = CDMOE
+    x = make_cdmoe_inputs(c["T"], c["hidden"], c["num_experts"], c["seed"], device=dev)
+    ws = dma.new_workspace(dma.dma_cdmoe_workspace_size(c["T"], c["num_experts"]), dev)
+    out = torch.empty_like(x["h"])
+
+    def step(i):
+        dma.dma_cdmoe_forward(x["h"], x["W_router"], x["down_embed"], x["up_embed"], c["top_k"], out=out,
+                              workspace=ws)
+
+    for i in range(warmup):
+        step(i)
+        flush.zero_()
+    assert dma.dma_check(ws) == 0
+    ranks_sync()
+    ms = run_steps(dma, step, 0, steps, flush)
+    ranks_sync()
+    split = run_steps(dma, step, steps, steps, flush, stages=True)
+    assert dma.dma_check(ws) == 0
+    n = len(split)
+    # bytes a token must move: its down and up expert rows, h in, the output out
+    row_bytes = c["T"] * (2 * c["top_k"] * c["hidden"] * 2 + 2 * c["hidden"] * 2)
+    router_flops = 2 * c["T"] * c["hidden"] * 2 * int(round(c["num_experts"] ** 0.5))
+    del x
+    return {"ms": sum(ms) / len(ms), "stage_ms": [sum(v[k] for v in split) / n for k in range(3)],
+            "bytes": row_bytes, "router_flops": router_flops, "launches": 2 * steps}
+
+
 def time_e2e(dma, wl, steps, warmup, dev):
     """Same metric through the public call with host (pinned) buffers: the H2D
     copy of every input and the D2H read of the output are inside each step.
@@ -475,6 +568,23 @@ def run_only(args):
     if args.batch:
         wl = wl.replace(B=args.batch)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    if args.backward:
+        r = time_backward(dma, wl, args.steps, args.warmup, flush, dev, torch.cuda.synchronize)
+        print(json.dumps({"workload": wl.name + " (backward)", "B": wl.B, "value": r["flops"] / (r["ms"] * 1e-3) / 1e12,
+                          "unit": "TFLOP/s", "ms_per_step": r["ms"], "stage_ms": r["stage_ms"],
+                          "gpu_launches": r["launches"]}), flush=True)
+        return
+    if args.cdmoe:
+        r = time_cdmoe(dma, args.steps, args.warmup, flush, dev, torch.cuda.synchronize)
+        print(json.dumps({"workload": "cdmoe", "value": CDMOE["T"] / (r["ms"] * 1e-3), "unit": "tokens/s",
+                          "ms_per_step": r["ms"], "stage_ms": r["stage_ms"],
+                          "expert_rows_gbs": r["bytes"] / (r["ms"] * 1e-3) / 1e9}), flush=True)
+        return
+    if args.prologue:
+        r = time_prologue(dma, wl, args.steps, args.warmup, flush, dev, torch.cuda.synchronize)
+        print(json.dumps({"workload": wl.name + " (prologue)", "B": wl.B, "value": r["bytes"] / (r["ms"] * 1e-3) / 1e9,
+                          "unit": "GB/s", "ms_per_step": r["ms"], "gpu_launches": r["launches"]}), flush=True)
+        return
     if args.cached:
         r = time_decode_cached(dma, wl, args.steps, args.warmup, flush, dev, torch.cuda.synchronize)
         line = {"workload": wl.name + " (cached dt)", "B": wl.B, "value": r["bytes"] / (r["ms"] * 1e-3) / 1e9,
@@ -572,6 +682,42 @@ def run_ours(args):
         result["gpu_launches"] += d["launches"]
         del d
         torch.cuda.empty_cache()
+        bw = time_backward(dma, WORKLOADS[HEADLINE], args.steps, args.warmup, flush, dev, ranks_sync)
+        bms = rank_max(bw["ms"])
+        others["backward_dense_eq"] = {
+            "value": round(aggregate_throughput(bw["flops"], bms, world) / 1e12, 3), "unit": "TFLOP/s",
+            "ms_per_step": round(bms, 5), "frac_of_bf16_peak": round(bw["flops"] / (bms * 1e-3) / 1e12 /
+                                                                      peaks["bf16_tflops"], 4),
+            "stage_ms": [round(x_, 5) for x_ in bw["stage_ms"]],
+            "note": "backward of the headline workload (selection held fixed): dt, kept-key lists, attention "
+                    "backward and dt chain; 10 d FLOPs per kept pair per query head"}
+        result["gpu_launches"] += bw["launches"]
+        del bw
+        torch.cuda.empty_cache()
+        cm = time_cdmoe(dma, args.steps, args.warmup, flush, dev, ranks_sync)
+        cms_ = rank_max(cm["ms"])
+        others["cdmoe"] = {"value": round(world * CDMOE["T"] / (cms_ * 1e-3), 1), "unit": "tokens/s",
+                           "ms_per_step": round(cms_, 5),
+                           "expert_rows_gbs": round(cm["bytes"] / (cms_ * 1e-3) / 1e9, 1),
+                           "frac_of_hbm": round(cm["bytes"] / (cms_ * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                           "router_tflops": round(cm["router_flops"] / (cm["stage_ms"][0] * 1e-3) / 1e12, 2)
+                           if cm["stage_ms"][0] > 0 else None,
+                           "stage_ms": [round(x_, 5) for x_ in cm["stage_ms"]],
+                           "config": dict(CDMOE)}
+        result["gpu_launches"] += cm["launches"]
+        del cm
+        torch.cuda.empty_cache()
+        pr = time_prologue(dma, WORKLOADS["long"], args.steps, args.warmup, flush, dev, ranks_sync)
+        pms = rank_max(pr["ms"])
+        others["prologue_long"] = {"value": round(world * pr["bytes"] / (pms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                                   "ms_per_step": round(pms, 5),
+                                   "frac_of_hbm": round(pr["bytes"] / (pms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                                   "bytes_per_step": pr["bytes"],
+                                   "note": "q/k RMSNorm + rotary embedding + KV-cache append of the long "
+                                           "workload's 32768 tokens"}
+        result["gpu_launches"] += pr["launches"]
+        del pr
+        torch.cuda.empty_cache()
         c = time_decode_cached(dma, WORKLOADS["decode"], args.steps, args.warmup, flush, dev, ranks_sync)
         cms = rank_max(c["ms"])
         others["decode_cached"] = {"value": round(world * c["bytes"] / (cms * 1e-3) / 1e9, 1), "unit": "GB/s",
@@ -641,6 +787,9 @@ def main():
     ap.add_argument("--only", choices=sorted(WORKLOADS), help="time one workload only (profiling)")
     ap.add_argument("--batch", type=int, default=0, help="with --only: override the batch size")
     ap.add_argument("--cached", action="store_true", help="with --only decode: incremental steps with cached dt")
+    ap.add_argument("--prologue", action="store_true", help="with --only: time the prologue on that geometry")
+    ap.add_argument("--backward", action="store_true", help="with --only: time the backward on that workload")
+    ap.add_argument("--cdmoe", action="store_true", help="with --only (any): time the CDMoE routing workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

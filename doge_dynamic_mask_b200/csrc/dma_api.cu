@@ -437,6 +437,145 @@ dma_status_t dma_decode_step_cached(const void* q, const void* k_cache, const vo
   return DMA_OK;
 }
 
+dma_status_t dma_prologue(const void* q, const void* k, const void* v, const float* q_norm_w,
+                          const float* k_norm_w, float eps, float rope_theta, const int32_t* positions, int B, int L,
+                          int Lmax, int Hq, int Hkv, int d, void* q_out, void* k_cache, void* v_cache,
+                          void* workspace, size_t ws_bytes, dma_stream_t stream) {
+  if (!q || !k || !v || !q_norm_w || !k_norm_w || !positions || !q_out || !k_cache || !v_cache || !workspace)
+    return DMA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_norm_w) || !aligned16(k_norm_w) ||
+      !aligned16(positions) || !aligned16(q_out) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(workspace))
+    return DMA_ERR_INVALID_ARG;
+  if (ws_bytes < kHeaderBytes) return DMA_ERR_WORKSPACE;
+  if (!(eps >= 0.0f && eps <= 1.0f) || !(rope_theta > 1.0f && rope_theta < 3.0e38f)) return DMA_ERR_INVALID_ARG;
+  if (L < 1 || Lmax < 1 || L > Lmax) return DMA_ERR_INVALID_ARG;
+  dma_status_t st = check_shape(B, Lmax, Hq, Hkv, d, 1);
+  if (st != DMA_OK) return st;
+  if (static_cast<long long>(B) * L * Hq >= (1LL << 31)) return DMA_ERR_UNSUPPORTED;
+  if ((st = device_ok()) != DMA_OK) return st;
+  const cudaError_t e = launch_prologue(q, k, v, q_norm_w, k_norm_w, eps, rope_theta, positions, B, L, Lmax, Hq, Hkv,
+                                        d, q_out, k_cache, v_cache, static_cast<uint32_t*>(workspace),
+                                        reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DMA_OK : cuda_fail(e);
+}
+
+// backward workspace: the prefill plan, then float32 dK, dV [B, L, Hkv, d],
+// d_dt [B, Hkv, L] and dx [B, L, Hkv]
+static size_t bwd_extra_off(const Geometry& g) { return align_up(prefill_plan_bytes(g), 256); }
+static size_t bwd_bytes(const Geometry& g) {
+  const size_t kv = static_cast<size_t>(g.B) * g.Lk * g.Hkv * g.d * 4;
+  const size_t per_key = static_cast<size_t>(g.B) * g.Hkv * g.Lk * 4;
+  return bwd_extra_off(g) + 2 * align_up(kv, 256) + 2 * align_up(per_key, 256);
+}
+
+size_t dma_backward_workspace_size(int B, int L, int Hq, int Hkv, int d, int keep_window_size) {
+  if (check_shape(B, L, Hq, Hkv, d, keep_window_size) != DMA_OK) return 0;
+  return bwd_bytes(Geometry{B, L, L, Hq, Hkv, d, keep_window_size});
+}
+
+dma_status_t dma_backward_prefill(const void* q, const void* k, const void* v, const float* W_dt, const float* A,
+                                  const int32_t* lengths, int B, int L, int Hq, int Hkv, int d, int keep_window_size,
+                                  float scale, const float* dt_in, const void* out, const void* dout, void* dq,
+                                  void* dk, void* dv, float* d_dt, float* dW_dt, float* dA, void* workspace,
+                                  size_t ws_bytes, dma_stream_t stream) {
+  if (!q || !k || !v || !W_dt || !A || !out || !dout || !dq || !dk || !dv || !dW_dt || !dA || !workspace)
+    return DMA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(W_dt) || !aligned16(A) || !aligned16(out) ||
+      !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dW_dt) ||
+      !aligned16(dA) || !aligned16(workspace) || (dt_in && !aligned16(dt_in)) || (d_dt && !aligned16(d_dt)) ||
+      (lengths && !aligned16(lengths)))
+    return DMA_ERR_INVALID_ARG;
+  if (!(scale >= 1.0e-20f && scale <= 1.0e20f)) return DMA_ERR_INVALID_ARG;
+  dma_status_t st = check_shape(B, L, Hq, Hkv, d, keep_window_size);
+  if (st != DMA_OK) return st;
+  if ((st = device_ok()) != DMA_OK) return st;
+  const Geometry g{B, L, L, Hq, Hkv, d, keep_window_size};
+  if (ws_bytes < bwd_bytes(g)) return DMA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t* err = static_cast<uint32_t*>(workspace);
+  const PrefillPlan plan = carve_prefill_plan(workspace, g);
+  char* base = static_cast<char*>(workspace) + bwd_extra_off(g);
+  const size_t kv = align_up(static_cast<size_t>(B) * L * Hkv * d * 4, 256);
+  const size_t per_key = align_up(static_cast<size_t>(B) * Hkv * L * 4, 256);
+  float* dk32 = reinterpret_cast<float*>(base);
+  float* dv32 = reinterpret_cast<float*>(base + kv);
+  float* ddt32 = reinterpret_cast<float*>(base + 2 * kv);
+  float* dx = reinterpret_cast<float*>(base + 2 * kv + per_key);
+  cudaError_t e;
+  const float* dt = dt_in;
+  if ((e = stage_mark(0, s)) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaMemsetAsync(base, 0, 2 * kv + per_key, s)) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaMemsetAsync(dW_dt, 0, static_cast<size_t>(Hkv) * d * Hkv * 4, s)) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaMemsetAsync(dA, 0, static_cast<size_t>(Hkv) * 4, s)) != cudaSuccess) return cuda_fail(e);
+  if (!dt) {
+    if ((e = launch_dt_scores(v, W_dt, A, B, L, Hkv, d, plan.dt, err, s)) != cudaSuccess) return cuda_fail(e);
+    dt = plan.dt;
+  }
+  if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e);
+  // the kept-key lists of every row tile (the forward's plan), built even when
+  // keep_window_size >= L (the lists then hold every visible key)
+  if ((e = launch_select_prefill(dt, lengths, g, plan, err, s)) != cudaSuccess) return cuda_fail(e);
+  if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e);
+  if ((e = launch_attn_backward(q, k, v, out, dout, g, scale, plan, dq, dk32, dv32, ddt32, err, s)) != cudaSuccess)
+    return cuda_fail(e);
+  if ((e = launch_dt_backward(v, W_dt, A, ddt32, dk32, dv32, B, L, Hkv, d, dx, dW_dt, dA, dk, dv, s)) != cudaSuccess)
+    return cuda_fail(e);
+  if (d_dt && (e = cudaMemcpyAsync(d_dt, ddt32, static_cast<size_t>(B) * Hkv * L * 4, cudaMemcpyDeviceToDevice, s)) !=
+                  cudaSuccess)
+    return cuda_fail(e);
+  if ((e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e);
+  return DMA_OK;
+}
+
+static int cdmoe_keys(int num_experts) {
+  for (int K = 16; K <= 128; K *= 2)
+    if (K * K == num_experts) return K;
+  return 0;
+}
+
+size_t dma_cdmoe_workspace_size(int T, int num_experts) {
+  const int K = cdmoe_keys(num_experts);
+  if (T < 1 || K == 0) return 0;
+  return kHeaderBytes + align_up(static_cast<size_t>(T) * 2 * K * 4, 256);
+}
+
+dma_status_t dma_cdmoe_forward(const void* h, const void* W_router, const void* down_embed, const void* up_embed,
+                               int T, int hidden, int num_experts, int top_k, const float* logits_in, void* out,
+                               int32_t* experts_out, float* scores_out, void* workspace, size_t ws_bytes,
+                               dma_stream_t stream) {
+  if (!h || !down_embed || !up_embed || !out || !workspace || (!logits_in && !W_router)) return DMA_ERR_INVALID_ARG;
+  if ((experts_out == nullptr) != (scores_out == nullptr)) return DMA_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(down_embed) || !aligned16(up_embed) || !aligned16(out) || !aligned16(workspace) ||
+      (W_router && !aligned16(W_router)) || (logits_in && !aligned16(logits_in)) ||
+      (experts_out && !aligned16(experts_out)) || (scores_out && !aligned16(scores_out)))
+    return DMA_ERR_INVALID_ARG;
+  if (T < 1 || hidden < 1 || top_k < 1) return DMA_ERR_INVALID_ARG;
+  const int K = cdmoe_keys(num_experts);
+  if (K == 0 || hidden % 64 != 0 || hidden > 8192 || top_k > K || top_k > 64) return DMA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(T) * hidden >= (1LL << 31)) return DMA_ERR_UNSUPPORTED;
+  if (ws_bytes < dma_cdmoe_workspace_size(T, num_experts)) return DMA_ERR_WORKSPACE;
+  dma_status_t st = device_ok();
+  if (st != DMA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t* err = static_cast<uint32_t*>(workspace);
+  const float* logits = logits_in;
+  cudaError_t e;
+  if ((e = stage_mark(0, s)) != cudaSuccess) return cuda_fail(e);
+  if (!logits) {
+    float* lg = reinterpret_cast<float*>(static_cast<char*>(workspace) + kHeaderBytes);
+    if ((e = launch_cdmoe_logits(h, W_router, T, hidden, K, lg, err, s)) != cudaSuccess) return cuda_fail(e);
+    logits = lg;
+  }
+  if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e);
+  if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e);
+  if ((e = launch_cdmoe_route_experts(h, logits, down_embed, up_embed, T, hidden, K, top_k, out, experts_out,
+                                      scores_out, s)) != cudaSuccess)
+    return cuda_fail(e);
+  if ((e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e);
+  return DMA_OK;
+}
+
 dma_status_t dma_check(void* workspace, int clear, dma_stream_t stream) {
   if (!workspace) return DMA_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -447,6 +586,7 @@ dma_status_t dma_check(void* workspace, int clear, dma_stream_t stream) {
   if (clear && word != 0 && (e = cudaMemset(workspace, 0, 4)) != cudaSuccess) return cuda_fail(e);
   if (word == kDevErrNone) return DMA_OK;
   if (word == kDevErrBadLength) return DMA_ERR_BAD_LENGTH;
+  if (word == kDevErrBadPosition) return DMA_ERR_BAD_POSITION;
   return DMA_ERR_TIMEOUT;
 }
 
@@ -465,6 +605,7 @@ const char* dma_status_string(dma_status_t status) {
     case DMA_ERR_CUDA: return "DMA_ERR_CUDA";
     case DMA_ERR_TIMEOUT: return "DMA_ERR_TIMEOUT";
     case DMA_ERR_BAD_LENGTH: return "DMA_ERR_BAD_LENGTH";
+    case DMA_ERR_BAD_POSITION: return "DMA_ERR_BAD_POSITION";
   }
   return "DMA_ERR_UNKNOWN";
 }

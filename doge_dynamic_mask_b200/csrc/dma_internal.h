@@ -27,6 +27,7 @@ constexpr long long kWaitLimitCycles = 2000000000LL;
 enum DeviceError : uint32_t {
   kDevErrNone = 0,
   kDevErrBadLength = 6,      // a lengths[b] outside [1, Lk]
+  kDevErrBadPosition = 7,    // a prologue token whose cache row is outside [0, Lmax)
   kDevErrTimeoutBase = 100,  // 100 + site: a bounded wait gave up
 };
 
@@ -145,6 +146,24 @@ cudaError_t launch_attn_decode(const void* q, const void* k, const void* v, cons
 cudaError_t launch_decode_update(const void* v_cache, const float* W, const float* A, const int32_t* lengths,
                                  const Geometry& g, const DecodePlan& plan, int32_t* done, int32_t* worst,
                                  uint32_t* err, cudaStream_t s);
+cudaError_t launch_prologue(const void* q, const void* k, const void* v, const float* q_w, const float* k_w,
+                            float eps, float theta, const int32_t* positions, int B, int L, int Lmax, int Hq, int Hkv,
+                            int d, void* q_out, void* k_cache, void* v_cache, uint32_t* err, cudaStream_t s);
+// CDMoE routing: router logits on the tensor cores (2K in {32, 64, 128, 256},
+// hidden a multiple of 64), then routing and experts (one CTA per token).
+cudaError_t launch_cdmoe_logits(const void* h, const void* W_router, int T, int hidden, int K, float* logits,
+                                uint32_t* err, cudaStream_t s);
+cudaError_t launch_cdmoe_route_experts(const void* h, const float* logits, const void* down_embed,
+                                       const void* up_embed, int T, int hidden, int K, int k, void* out,
+                                       int32_t* experts_out, float* scores_out, cudaStream_t s);
+// backward: attention with the selection held fixed (float32 dK / dV / d_dt
+// accumulators, zeroed by the caller), then the dt chain (dk / dv to bf16, dW, dA)
+cudaError_t launch_attn_backward(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                                 const Geometry& g, float scale, const PrefillPlan& plan, void* dq, float* dk32,
+                                 float* dv32, float* ddt32, uint32_t* err, cudaStream_t s);
+cudaError_t launch_dt_backward(const void* v, const float* W, const float* A, const float* ddt32, const float* dk32,
+                               const float* dv32, int B, int L, int Hkv, int d, float* dx, float* dW, float* dA,
+                               void* dk, void* dv, cudaStream_t s);
 cudaError_t launch_decode_state_finish(const int32_t* lengths, const Geometry& g, const DecodePlan& plan,
                                        int32_t* done, int32_t* worst, cudaStream_t s);
 

@@ -1,0 +1,149 @@
+// Prologue of the attention forward: q_norm / k_norm, rotary embedding, KV-cache append.
+//
+// Method: page "Transformers 中的 Doge 小语言模型完全指南", section
+// "动态掩码注意力（DMA）：从缓存 value states 生成稀疏掩码", forward-chain steps 1 and 2:
+// after the projections, Q and K pass an RMSNorm over head_dim (q_norm / k_norm,
+// the Llama RMSNorm the section "从源码理解两大核心模块" says Doge reuses), then
+// the rotary position embedding (Llama's apply_rotary_pos_emb); K and V are then
+// appended to the KV cache.  rms_norm_eps comes from "DogeConfig 全参数详解".
+//
+//   y_c   = w_c * x_c / sqrt(mean_c(x^2) + eps)                  (per head row of d channels)
+//   out_i = y_i cos(a_i) - y_{i+d/2} sin(a_i),  out_{i+d/2} = y_{i+d/2} cos(a_i) + y_i sin(a_i)
+//   a_i   = pos * theta^(-2i/d),  i < d/2,  pos = positions[b] + t
+//
+// Design.  Memory-bound: every projected row is read once and written once.
+// One CTA per token: the d/2 angles of its position are formed in double
+// precision (a position of 10^5 times a frequency near 1 would lose about
+// 2^-7 rad of its angle in float32, the size of a bf16 rounding) and their
+// cosines and sines kept in shared memory; then each group of d/8 lanes owns
+// one head row as sixteen-byte vectors (eight bf16 channels per lane): the
+// mean square is a group shuffle reduction, and channel i's rotation partner
+// i + d/2 sits in the lane d/16 positions away, one shuffle.  Arithmetic is
+// float32 with one rounding to bf16 at the end; V rows are copied bit for bit.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace dma {
+namespace {
+
+constexpr int kPrologueThreads = 128;
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float* f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPrologueThreads)
+    prologue_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k, const uint4* __restrict__ v,
+                    const float* __restrict__ q_w, const float* __restrict__ k_w, float eps, double log_theta,
+                    const int32_t* __restrict__ positions, int L, int Lmax, int Hq, int Hkv,
+                    uint4* __restrict__ q_out, uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                    uint32_t* err) {
+  constexpr int kLanesPerRow = D / 8;               // 16-byte vectors per head row
+  constexpr int kRowsPerWarp = 32 / kLanesPerRow;
+  constexpr int kHalf = kLanesPerRow / 2;           // lane distance of channel i's partner i + d/2
+  __shared__ float s_cos[D / 2], s_sin[D / 2];
+
+  const int token = blockIdx.x;                     // b * L + t
+  const int b = token / L, t = token - b * L;
+  const int pos = positions[b] + t;
+  const bool in_cache = positions[b] >= 0 && pos < Lmax;
+  if (threadIdx.x == 0 && !in_cache) raise_error(err, kDevErrBadPosition);
+  if (threadIdx.x < D / 2) {
+    // theta^(-2i/d) and the angle in double precision, then its cosine and sine
+    const double inv_freq = exp(-2.0 * static_cast<double>(threadIdx.x) / D * log_theta);
+    double sn, cs;
+    sincos(static_cast<double>(pos) * inv_freq, &sn, &cs);
+    s_cos[threadIdx.x] = static_cast<float>(cs);
+    s_sin[threadIdx.x] = static_cast<float>(sn);
+  }
+  __syncthreads();
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane % kLanesPerRow;              // this lane's 8 channels: [8 sub, 8 sub + 8)
+  const int rows = Hq + 2 * Hkv;                    // q heads, then k heads, then v heads
+  const size_t qrow0 = static_cast<size_t>(token) * Hq;
+  const size_t krow0 = static_cast<size_t>(token) * Hkv;
+  const size_t crow0 = (static_cast<size_t>(b) * Lmax + pos) * Hkv;
+  for (int base = warp * kRowsPerWarp; base < rows; base += (kPrologueThreads / 32) * kRowsPerWarp) {
+    const int r = base + lane / kLanesPerRow;
+    const bool live = r < rows;
+    const bool is_q = r < Hq, is_k = !is_q && r < Hq + Hkv;
+    uint4 u = make_uint4(0u, 0u, 0u, 0u);
+    if (live) {
+      if (is_q) u = q[(qrow0 + r) * kLanesPerRow + sub];
+      else if (is_k) u = k[(krow0 + (r - Hq)) * kLanesPerRow + sub];
+      else u = v[(krow0 + (r - Hq - Hkv)) * kLanesPerRow + sub];
+    }
+    if (live && !is_q && !is_k) {
+      if (in_cache) v_cache[(crow0 + (r - Hq - Hkv)) * kLanesPerRow + sub] = u;   // V: appended as is
+    }
+    // the shuffles below run on every lane of the warp (uniform trip count)
+    float x[8];
+    bf16x8_to_f32(u, x);
+    float ss = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+#pragma unroll
+    for (int o = kLanesPerRow / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+    const float inv = 1.0f / sqrtf(ss * (1.0f / D) + eps);
+    const float* w = is_q ? q_w : k_w;
+    float y[8], yp[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] = (live && (is_q || is_k)) ? w[8 * sub + e] * (x[e] * inv) : 0.0f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) yp[e] = __shfl_xor_sync(0xFFFFFFFFu, y[e], kHalf);
+    if (live && (is_q || is_k)) {
+      const bool low = sub < kHalf;                 // channels below d/2
+      const int i0 = 8 * (low ? sub : sub - kHalf); // pair index of this lane's first channel
+      uint32_t pk[4];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        float o0, o1;
+        if (low) {
+          o0 = y[e] * s_cos[i0 + e] - yp[e] * s_sin[i0 + e];
+          o1 = y[e + 1] * s_cos[i0 + e + 1] - yp[e + 1] * s_sin[i0 + e + 1];
+        } else {
+          o0 = y[e] * s_cos[i0 + e] + yp[e] * s_sin[i0 + e];
+          o1 = y[e + 1] * s_cos[i0 + e + 1] + yp[e + 1] * s_sin[i0 + e + 1];
+        }
+        pk[e / 2] = pack_bf16x2(o0, o1);
+      }
+      const uint4 o = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      if (is_q) q_out[(qrow0 + r) * kLanesPerRow + sub] = o;
+      else if (in_cache) k_cache[(crow0 + (r - Hq)) * kLanesPerRow + sub] = o;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_prologue(const void* q, const void* k, const void* v, const float* q_w, const float* k_w,
+                            float eps, float theta, const int32_t* positions, int B, int L, int Lmax, int Hq, int Hkv,
+                            int d, void* q_out, void* k_cache, void* v_cache, uint32_t* err, cudaStream_t s) {
+  const long long tokens = static_cast<long long>(B) * L;
+  if (tokens > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  const double log_theta = log(static_cast<double>(theta));
+  const dim3 grid(static_cast<unsigned>(tokens)), block(kPrologueThreads);
+  if (d == 64)
+    prologue_kernel<64><<<grid, block, 0, s>>>(
+        static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v), q_w, k_w, eps,
+        log_theta, positions, L, Lmax, Hq, Hkv, static_cast<uint4*>(q_out), static_cast<uint4*>(k_cache),
+        static_cast<uint4*>(v_cache), err);
+  else if (d == 128)
+    prologue_kernel<128><<<grid, block, 0, s>>>(
+        static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v), q_w, k_w, eps,
+        log_theta, positions, L, Lmax, Hq, Hkv, static_cast<uint4*>(q_out), static_cast<uint4*>(k_cache),
+        static_cast<uint4*>(v_cache), err);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+}  // namespace dma

@@ -97,7 +97,7 @@ __device__ __forceinline__ uint32_t find_bin_from_top(const uint32_t* hist, int 
 }
 
 // k-th largest (1-based) of n distinct keys held in shared memory.
-__device__ __noinline__ uint64_t select_kth_smem(const uint64_t* keys, int n, uint32_t k, SelScratch sc) {
+static __device__ __noinline__ uint64_t select_kth_smem(const uint64_t* keys, int n, uint32_t k, SelScratch sc) {
   uint64_t vor = 0, vand = ~0ull;
   for (int e = threadIdx.x; e < n; e += blockDim.x) {
     vor |= keys[e];
@@ -137,7 +137,7 @@ __device__ __noinline__ uint64_t select_kth_smem(const uint64_t* keys, int n, ui
 }
 
 // Index of the k-th (1-based) position j in [0, n) with bits[j] == val, in increasing j.
-__device__ __noinline__ int kth_matching_index(const uint32_t* __restrict__ bits, int n, uint32_t val, uint32_t k,
+static __device__ __noinline__ int kth_matching_index(const uint32_t* __restrict__ bits, int n, uint32_t val, uint32_t k,
                                                SelScratch sc) {
   const uint32_t lane = lane_id(), warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const int seg = ((n + nw - 1) / nw + 31) / 32 * 32;
@@ -224,7 +224,7 @@ __device__ __forceinline__ void row_for_each(const uint32_t* __restrict__ bits, 
 }
 
 // k-th largest composite key (1 <= k <= n) among positions [0, n) of a dt row.
-__device__ __noinline__ uint64_t select_kth_global(const uint32_t* __restrict__ bits, int n, uint32_t k,
+static __device__ __noinline__ uint64_t select_kth_global(const uint32_t* __restrict__ bits, int n, uint32_t k,
                                                    SelScratch sc) {
   uint32_t vor = 0u, vand = ~0u;
   row_for_each(bits, n, [&](uint32_t b, int, bool ok) {

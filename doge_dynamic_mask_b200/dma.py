@@ -22,7 +22,7 @@ _lib = ctypes.CDLL(_LIB_PATH)
 
 DMA_OK = 0
 STATUS = {0: "DMA_OK", 1: "DMA_ERR_INVALID_ARG", 2: "DMA_ERR_UNSUPPORTED", 3: "DMA_ERR_WORKSPACE",
-          4: "DMA_ERR_CUDA", 5: "DMA_ERR_TIMEOUT", 6: "DMA_ERR_BAD_LENGTH"}
+          4: "DMA_ERR_CUDA", 5: "DMA_ERR_TIMEOUT", 6: "DMA_ERR_BAD_LENGTH", 7: "DMA_ERR_BAD_POSITION"}
 
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 _lib.dma_workspace_size.restype = _sz
@@ -42,6 +42,16 @@ _lib.dma_decode_state_init.restype = _i
 _lib.dma_decode_state_init.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
 _lib.dma_decode_step_cached.restype = _i
 _lib.dma_decode_step_cached.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _sz, _vp]
+_lib.dma_prologue.restype = _i
+_lib.dma_prologue.argtypes = [_vp] * 5 + [_f, _f, _vp] + [_i] * 6 + [_vp] * 4 + [_sz, _vp]
+_lib.dma_cdmoe_workspace_size.restype = _sz
+_lib.dma_cdmoe_workspace_size.argtypes = [_i, _i]
+_lib.dma_cdmoe_forward.restype = _i
+_lib.dma_cdmoe_forward.argtypes = [_vp] * 4 + [_i] * 4 + [_vp] * 5 + [_sz, _vp]
+_lib.dma_backward_workspace_size.restype = _sz
+_lib.dma_backward_workspace_size.argtypes = [_i] * 6
+_lib.dma_backward_prefill.restype = _i
+_lib.dma_backward_prefill.argtypes = [_vp] * 6 + [_i] * 6 + [_f] + [_vp] * 10 + [_sz, _vp]
 _lib.dma_selftest_wait.restype = _i
 _lib.dma_selftest_wait.argtypes = [_vp, _vp]
 _lib.dma_check.restype = _i
@@ -144,6 +154,76 @@ def dma_decode_step(q, k_cache, v_cache, W_dt, A, lengths, keep_window_size, sca
                              Hkv, d, keep_window_size, float(scale), _ptr(dt_in), _ptr(out), _ptr(workspace),
                              workspace.numel(), _stream(stream)),
         "dma_decode_step")
+    return out
+
+
+def dma_prologue(q, k, v, q_norm_w, k_norm_w, positions, k_cache, v_cache, eps=1e-6, rope_theta=10000.0,
+                 q_out=None, workspace=None, stream=None):
+    """q/k RMSNorm over head_dim, rotary embedding, and the KV-cache append of
+    L new tokens per sequence (token t of sequence b at cache row positions[b] + t).
+    Returns q_out; k_cache and v_cache are written in place."""
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    Lmax = k_cache.shape[1]
+    if q_out is None:
+        q_out = torch.empty_like(q)
+    if workspace is None:
+        workspace = new_workspace(256, q.device)
+    _ok(_lib.dma_prologue(_ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), float(eps), float(rope_theta),
+                          _ptr(positions), B, L, Lmax, Hq, Hkv, d, _ptr(q_out), _ptr(k_cache), _ptr(v_cache),
+                          _ptr(workspace), workspace.numel(), _stream(stream)),
+        "dma_prologue")
+    return q_out
+
+
+def dma_backward_workspace_size(B, L, Hq, Hkv, d, keep_window_size) -> int:
+    return int(_lib.dma_backward_workspace_size(B, L, Hq, Hkv, d, keep_window_size))
+
+
+def dma_backward_prefill(q, k, v, W_dt, A, lengths, keep_window_size, out, dout, scale=None, dt_in=None,
+                         workspace=None, want_d_dt=False, stream=None):
+    """Gradients of sum(out * dout) with the selection held fixed: returns
+    (dq, dk, dv) bf16, dW_dt and dA float32, and d_dt [B, Hkv, L] float32 when
+    want_d_dt."""
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = d ** -0.5
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dW = torch.empty_like(W_dt)
+    dA = torch.empty_like(A)
+    d_dt = torch.empty((B, Hkv, L), dtype=torch.float32, device=q.device) if want_d_dt else None
+    if workspace is None:
+        workspace = new_workspace(dma_backward_workspace_size(B, L, Hq, Hkv, d, keep_window_size), q.device)
+    _ok(_lib.dma_backward_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(W_dt), _ptr(A), _ptr(lengths), B, L, Hq, Hkv, d,
+                                  keep_window_size, float(scale), _ptr(dt_in), _ptr(out), _ptr(dout), _ptr(dq),
+                                  _ptr(dk), _ptr(dv), _ptr(d_dt), _ptr(dW), _ptr(dA), _ptr(workspace),
+                                  workspace.numel(), _stream(stream)),
+        "dma_backward_prefill")
+    return (dq, dk, dv, dW, dA, d_dt) if want_d_dt else (dq, dk, dv, dW, dA)
+
+
+def dma_cdmoe_workspace_size(T, num_experts) -> int:
+    return int(_lib.dma_cdmoe_workspace_size(T, num_experts))
+
+
+def dma_cdmoe_forward(h, W_router, down_embed, up_embed, top_k, logits_in=None, out=None, experts_out=None,
+                      scores_out=None, workspace=None, stream=None):
+    """Routed CDMoE output [T, hidden] (bf16).  With experts_out / scores_out
+    ([T, top_k] int32 / float32) the kept experts are written too, best first."""
+    T, hidden = h.shape
+    num_experts = down_embed.shape[0]
+    if out is None:
+        out = torch.empty_like(h)
+    if workspace is None:
+        size = dma_cdmoe_workspace_size(T, num_experts)
+        if size == 0:
+            raise ValueError("unsupported CDMoE geometry")
+        workspace = new_workspace(size, h.device)
+    _ok(_lib.dma_cdmoe_forward(_ptr(h), _ptr(W_router), _ptr(down_embed), _ptr(up_embed), T, hidden, num_experts,
+                               top_k, _ptr(logits_in), _ptr(out), _ptr(experts_out), _ptr(scores_out),
+                               _ptr(workspace), workspace.numel(), _stream(stream)),
+        "dma_cdmoe_forward")
     return out
 
 

@@ -107,3 +107,46 @@ def make_inputs(wl: Workload, device="cpu", seed: Optional[int] = None):
 def shrink(wl: Workload, **kw) -> Workload:
     """A smaller variant of a workload (same value recipe) for tests."""
     return wl.replace(name=wl.name + "_small", **kw)
+
+
+def make_prologue_inputs(B, L, Lmax, Hq, Hkv, d, seed, device="cpu", positions=None):
+    """Inputs of the prologue (q/k RMSNorm, rotary embedding, KV-cache append):
+    projected q [B,L,Hq,d], k/v [B,L,Hkv,d] and caches [B,Lmax,Hkv,d] ~ N(0,1)
+    rounded to bf16; RMSNorm weights [d] ~ U[0.5, 1.5] float32 (a learned
+    scale around its initial value 1); positions [B] int32 ~ U[0, Lmax - L]
+    unless given.  Draw order: q, k, v, q_norm_w, k_norm_w, positions,
+    k_cache, v_cache."""
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    q = _randn_bf16((B, L, Hq, d), gen, device, chunk_rows=1)
+    k = _randn_bf16((B, L, Hkv, d), gen, device, chunk_rows=1)
+    v = _randn_bf16((B, L, Hkv, d), gen, device, chunk_rows=1)
+    q_w = torch.rand((d,), generator=gen, device=device, dtype=torch.float32) + 0.5
+    k_w = torch.rand((d,), generator=gen, device=device, dtype=torch.float32) + 0.5
+    pos = torch.randint(0, Lmax - L + 1, (B,), generator=gen, device=device, dtype=torch.int64).to(torch.int32)
+    if positions is not None:
+        pos = torch.as_tensor(positions, dtype=torch.int32, device=device)
+    k_cache = _randn_bf16((B, Lmax, Hkv, d), gen, device, chunk_rows=1)
+    v_cache = _randn_bf16((B, Lmax, Hkv, d), gen, device, chunk_rows=1)
+    return {"q": q, "k": k, "v": v, "q_w": q_w, "k_w": k_w, "positions": pos, "k_cache": k_cache,
+            "v_cache": v_cache}
+
+
+def make_cdmoe_inputs(T, hidden, num_experts, seed, device="cpu"):
+    """Inputs of the CDMoE routing: hidden states h [T, hidden] ~ N(0, 1) and
+    the router weight W_router [2K, hidden] (K = sqrt(num_experts)) ~ N(0, 0.02)
+    plus the expert tables down_embed / up_embed [num_experts, hidden]
+    ~ N(0, 0.02) (the models' initializer_range), all rounded to bf16.
+    Draw order: h, W_router, down_embed, up_embed."""
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    K = int(round(num_experts ** 0.5))
+    h = _randn_bf16((T, hidden), gen, device)
+    w = (torch.randn((2 * K, hidden), generator=gen, device=device, dtype=torch.float32) * 0.02).to(torch.bfloat16)
+    down = (torch.randn((num_experts, hidden), generator=gen, device=device, dtype=torch.float32) * 0.02).to(
+        torch.bfloat16)
+    up = (torch.randn((num_experts, hidden), generator=gen, device=device, dtype=torch.float32) * 0.02).to(
+        torch.bfloat16)
+    return {"h": h, "W_router": w, "down_embed": down, "up_embed": up}

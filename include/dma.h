@@ -64,7 +64,8 @@ typedef enum {
   DMA_ERR_WORKSPACE = 3,   /* workspace smaller than dma_workspace_size() */
   DMA_ERR_CUDA = 4,        /* a CUDA call failed; dma_last_cuda_error() has the code */
   DMA_ERR_TIMEOUT = 5,     /* a bounded device wait gave up (reported by dma_check) */
-  DMA_ERR_BAD_LENGTH = 6   /* a lengths[b] outside [1, Lk] (reported by dma_check; clamped) */
+  DMA_ERR_BAD_LENGTH = 6,  /* a lengths[b] outside [1, Lk] (reported by dma_check; clamped) */
+  DMA_ERR_BAD_POSITION = 7 /* a prologue token outside the cache (reported by dma_check; not written) */
 } dma_status_t;
 
 /*
@@ -157,6 +158,92 @@ DMA_API dma_status_t dma_decode_step(const void* q, const void* k_cache, const v
                              const float* A, const int32_t* lengths, int B, int Lk, int Hq, int Hkv, int d,
                              int keep_window_size, float scale, const float* dt_in, void* out, void* workspace,
                              size_t ws_bytes, dma_stream_t stream);
+
+/*
+ * Prologue, [DMA steps 1-2]: the steps of the attention forward between the
+ * projections and the dynamic mask, for L new tokens per sequence.  Q and K
+ * each pass an RMSNorm over head_dim (q_norm / k_norm: Llama's RMSNorm, which
+ * the page says Doge reuses) and then the rotary position embedding (Llama's
+ * pairing of channel i with channel i + d/2); K and V are appended to the
+ * cache (past_key_values.update).  For token t of sequence b, pos = positions[b] + t:
+ *   y_c        = w_c * x_c / sqrt(mean over the d channels of x^2 + eps)
+ *   a_i        = pos * rope_theta^(-2i/d),  i < d/2
+ *   out_i      = y_i cos a_i - y_{i+d/2} sin a_i
+ *   out_{i+d/2} = y_{i+d/2} cos a_i + y_i sin a_i
+ * computed in float32 (angles in double precision) and rounded once to bf16.
+ *   q, k, v        [B, L, Hq, d], [B, L, Hkv, d], [B, L, Hkv, d] bf16 projected states
+ *   q_norm_w, k_norm_w  [d] float32 RMSNorm weights;  eps: rms_norm_eps ([Config]: 1e-6)
+ *   rope_theta     > 1 (the page gives no default; Llama's is 10000)
+ *   positions      [B] int32 (device): cache row of each sequence's first new token
+ *   q_out          [B, L, Hq, d] bf16 (written)
+ *   k_cache, v_cache [B, Lmax, Hkv, d] bf16: rows positions[b] .. positions[b] + L - 1
+ *                  are written (normalised and rotated K; V as given); other rows untouched
+ *   workspace      >= 256 bytes, zeroed once: its status word records a token whose
+ *                  cache row lies outside [0, Lmax) (DMA_ERR_BAD_POSITION via dma_check);
+ *                  such a token's q_out row is still written, its cache rows are not.
+ * Supported: d in {64, 128}, Hq a multiple of Hkv, Hkv <= 16, Hq / Hkv <= 8.
+ */
+DMA_API dma_status_t dma_prologue(const void* q, const void* k, const void* v, const float* q_norm_w,
+                                  const float* k_norm_w, float eps, float rope_theta, const int32_t* positions,
+                                  int B, int L, int Lmax, int Hq, int Hkv, int d, void* q_out, void* k_cache,
+                                  void* v_cache, void* workspace, size_t ws_bytes, dma_stream_t stream);
+
+/*
+ * Backward of S1 + S2 + S3 ([DMA step 3] closing paragraph: dt is learnt end
+ * to end from the value states; [DMA step 4]).  The top-k selection has no
+ * gradient: each row's kept set is held fixed, and the gradient reaches dt
+ * through the kept keys' bias.  For the loss sum(out * dout):
+ *   dP = dO V^T, D_i = dO_i . O_i, dS = P (dP - D),
+ *   dq = scale dS K, dk = scale dS^T Q, dv = P^T dO + (dt path),
+ *   d_dt[b, g, j] = sum over the group's heads and rows of dS[., j],
+ *   dt = exp(A softplus(x)), x = v_flat W_dt:
+ *   dA = sum d_dt dt softplus(x), dx = d_dt dt A sigmoid(x),
+ *   dW_dt = v_flat^T dx, dv_flat += dx W_dt^T.
+ * Arguments as dma_forward_prefill, plus:
+ *   out      [B, L, Hq, d] bf16: the forward's output for the same inputs
+ *   dout     [B, L, Hq, d] bf16: the gradient of the loss with respect to out
+ *   dq       [B, L, Hq, d] bf16 (written);  dk, dv [B, L, Hkv, d] bf16 (written)
+ *   d_dt     [B, Hkv, L] float32 (written) or NULL
+ *   dW_dt    [Hkv*d, Hkv] float32 (written);  dA [Hkv] float32 (written)
+ *   dt_in    as in the forward (NULL: dt computed from W_dt and A); the dt chain
+ *            always starts from W_dt and A, which are required.
+ *   workspace  dma_backward_workspace_size(...) bytes, zeroed once (status word first).
+ * The accumulations (dk, dv, d_dt, dW_dt, dA) add float32 partial sums in an
+ * unspecified order, so results may differ in the last bits between calls.
+ */
+DMA_API size_t dma_backward_workspace_size(int B, int L, int Hq, int Hkv, int d, int keep_window_size);
+DMA_API dma_status_t dma_backward_prefill(const void* q, const void* k, const void* v, const float* W_dt,
+                                          const float* A, const int32_t* lengths, int B, int L, int Hq, int Hkv,
+                                          int d, int keep_window_size, float scale, const float* dt_in,
+                                          const void* out, const void* dout, void* dq, void* dk, void* dv,
+                                          float* d_dt, float* dW_dt, float* dA, void* workspace, size_t ws_bytes,
+                                          dma_stream_t stream);
+
+/*
+ * CDMoE routing ([CDMoE], section "跨域 MoE（CDMoE）" of the same page): the
+ * routed experts of the Cross Domain Mixture of Experts for T tokens.
+ * router_gate maps each hidden state to 2K logits (K = num_keys =
+ * floor(sqrt(num_experts))): columns [0, K) are domain x, [K, 2K) domain y.
+ * Each domain keeps its top_k best keys (ties: lower key index); pair (a, b)
+ * of the two kept sets scores s_x[a] + s_y[b] (float32) and names expert
+ * a * K + b; the token keeps the top_k best pairs (ties: lower expert index),
+ * weights them by the softmax of their scores, and adds
+ *   out = sum_e w_e * silu(h . down_embed[e]) * up_embed[e].
+ *   h            [T, hidden] bf16 hidden states
+ *   W_router     [2K, hidden] bf16 router_gate weight (the Linear layout: one row per logit), no bias
+ *   down_embed, up_embed  [num_experts, hidden] bf16 expert tables
+ *   num_experts  K * K with K in {16, 32, 64, 128};  top_k in [1, min(K, 64)]
+ *   hidden       a multiple of 64, at most 8192
+ *   logits_in    [T, 2K] float32 or NULL: when given, the router GEMM is skipped
+ *   out          [T, hidden] bf16 (written): the routed part, to be added to the shared expert's output
+ *   experts_out, scores_out  [T, top_k] int32 / float32 or both NULL: the kept experts, best first
+ *   workspace    dma_cdmoe_workspace_size(T, num_experts) bytes, zeroed once (status word first)
+ */
+DMA_API size_t dma_cdmoe_workspace_size(int T, int num_experts);
+DMA_API dma_status_t dma_cdmoe_forward(const void* h, const void* W_router, const void* down_embed,
+                                       const void* up_embed, int T, int hidden, int num_experts, int top_k,
+                                       const float* logits_in, void* out, int32_t* experts_out, float* scores_out,
+                                       void* workspace, size_t ws_bytes, dma_stream_t stream);
 
 /*
  * Incremental decode with cached dt.  dt is one linear projection per cached

@@ -130,3 +130,62 @@ def test_cached_decode_state_size_and_argument_errors(lib):
     assert step(*a) == 1
     a = list(args); a[8] = 6; a[9] = 4
     assert step(*a) == 1
+
+
+def test_prologue_argument_errors(lib):
+    vp = ctypes.c_void_p
+    p16 = vp(1 << 20)          # aligned dummy address, never dereferenced
+    bad = vp((1 << 20) + 4)    # misaligned
+    f = lib.dma_prologue
+    f.restype = ctypes.c_int
+    f.argtypes = [vp] * 5 + [ctypes.c_float, ctypes.c_float, vp] + [ctypes.c_int] * 6 + [vp] * 4 + [
+        ctypes.c_size_t, vp]
+    args = [p16] * 5 + [1e-6, 10000.0, p16, 2, 16, 64, 8, 4, 64, p16, p16, p16, p16, 256, None]
+    a = list(args); a[0] = None
+    assert f(*a) == 1                            # DMA_ERR_INVALID_ARG
+    a = list(args); a[3] = bad
+    assert f(*a) == 1
+    a = list(args); a[7] = None                  # positions are required
+    assert f(*a) == 1
+    a = list(args); a[18] = 255
+    assert f(*a) == 3                            # DMA_ERR_WORKSPACE: no room for the status word
+    a = list(args); a[9] = 65
+    assert f(*a) == 1                            # L > Lmax
+    a = list(args); a[6] = 1.0
+    assert f(*a) == 1                            # rope_theta must exceed 1
+    a = list(args); a[5] = float("nan")
+    assert f(*a) == 1
+    a = list(args); a[13] = 96
+    assert f(*a) == 2                            # d not supported
+    a = list(args); a[11] = 6
+    assert f(*a) == 1                            # Hq % Hkv != 0
+    lib.dma_status_string.restype = ctypes.c_char_p
+    assert lib.dma_status_string(7) == b"DMA_ERR_BAD_POSITION"
+
+
+def test_cdmoe_workspace_and_argument_errors(lib):
+    vp = ctypes.c_void_p
+    p16 = vp(1 << 20)          # aligned dummy address, never dereferenced
+    size = lib.dma_cdmoe_workspace_size
+    size.restype = ctypes.c_size_t
+    size.argtypes = [ctypes.c_int, ctypes.c_int]
+    assert size(100, 16384) == 256 + ((100 * 256 * 4 + 255) // 256) * 256      # header + float32 logits
+    assert size(100, 1000) == 0                                                  # not a square of 16..128
+    f = lib.dma_cdmoe_forward
+    f.restype = ctypes.c_int
+    f.argtypes = [vp] * 4 + [ctypes.c_int] * 4 + [vp] * 5 + [ctypes.c_size_t, vp]
+    args = [p16] * 4 + [8, 1024, 16384, 64] + [None, p16, None, None, p16, 1 << 20, None]
+    a = list(args); a[0] = None
+    assert f(*a) == 1
+    a = list(args); a[1] = None                       # no router weight and no logits
+    assert f(*a) == 1
+    a = list(args); a[10] = p16                       # experts_out without scores_out
+    assert f(*a) == 1
+    a = list(args); a[7] = 65
+    assert f(*a) == 2                                 # top_k above 64
+    a = list(args); a[6] = 1000
+    assert f(*a) == 2                                 # num_experts not K * K
+    a = list(args); a[5] = 1000
+    assert f(*a) == 2                                 # hidden not a multiple of 64
+    a = list(args); a[13] = 100
+    assert f(*a) == 3                                 # workspace too small

@@ -1,0 +1,81 @@
+"""Parity of the backward (through the C ABI) with the float64 oracle, the
+kept-key selection held fixed and built from the same float32 dt (the
+oracle's, passed as dt_in).  The forward output the backward takes is the
+oracle's, rounded to bf16.
+
+Bars (derived from the arithmetic): the kernels round P and dS to bf16 for
+the tensor core (relative error 2^-9 each, accumulated in float32 over up to
+a few thousand keys or rows with mixed signs) and round dq, dk, dv to bf16;
+every gradient G must satisfy
+  max |got - want| <= 2e-2 * max |want|   and   mean |got - want| <= 4e-3 * mean |want|.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from doge_dynamic_mask_b200.workloads import Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+MAX_REL, MEAN_REL = 2e-2, 4e-3
+
+
+@pytest.fixture(scope="module")
+def dma():
+    from doge_dynamic_mask_b200 import build
+    build.build()
+    from doge_dynamic_mask_b200 import dma as m
+    return m
+
+
+def f64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def assert_grad_close(got, want, what):
+    g = f64(got) if isinstance(got, torch.Tensor) else np.asarray(got, np.float64)
+    assert np.isfinite(g).all(), what
+    err = np.abs(g - want)
+    scale_max, scale_mean = np.abs(want).max(), np.abs(want).mean()
+    assert err.max() <= MAX_REL * scale_max and err.mean() <= MEAN_REL * scale_mean, (
+        f"{what}: max {err.max():.3e} (bar {MAX_REL * scale_max:.3e}), mean {err.mean():.3e} "
+        f"(bar {MEAN_REL * scale_mean:.3e})")
+
+
+def run_case(dma, wl, dout_seed=1):
+    x = make_inputs(wl)
+    q, k, v = f64(x["q"]), f64(x["k"]), f64(x["v"])
+    W, A = x["W"].double().numpy(), x["A"].double().numpy()
+    lengths = x["lengths"].numpy()
+    dt = oracle.dt_scores(v, W, A)
+    out = oracle.prefill(q, k, v, W, A, lengths, wl.w, wl.scale, dt=dt)
+    g = torch.Generator().manual_seed(dout_seed)
+    dout = torch.randn(x["q"].shape, generator=g).to(torch.bfloat16)
+    want = oracle.prefill_backward(q, k, v, W, A, lengths, wl.w, wl.scale, f64(dout), dt_fixed=dt)
+    d = {n: t.cuda() for n, t in x.items()}
+    got = dma.dma_backward_prefill(d["q"], d["k"], d["v"], d["W"], d["A"], d["lengths"], wl.w,
+                                   torch.from_numpy(out).to(torch.bfloat16).cuda(), dout.cuda(),
+                                   dt_in=torch.from_numpy(dt).cuda(), want_d_dt=True)
+    torch.cuda.synchronize()
+    names = ("dq", "dk", "dv", "dW", "dA", "d_dt")
+    order = (0, 1, 2, 4, 5, 3)    # oracle returns dq, dk, dv, d_dt, dW, dA
+    for name, gi, wi in zip(names, range(6), order):
+        assert_grad_close(got[gi], want[wi], name)
+
+
+def wl(B, L, Hq, Hkv, d, w, lens=None, seed=0):
+    lo, hi = (None, None) if lens is None else lens
+    return Workload("bwd", "prefill", B=B, L=L, Hq=Hq, Hkv=Hkv, d=d, w=w, a_lo=-2.0, a_hi=-0.1, seed=seed,
+                    len_lo=lo, len_hi=hi)
+
+
+@pytest.mark.parametrize("case", [
+    wl(1, 200, 4, 2, 64, 64, seed=1),              # top-k active, ragged row tile
+    wl(2, 130, 2, 2, 64, 1000, seed=2),            # window >= L: causal + bias
+    wl(2, 300, 6, 2, 64, 96, lens=(150, 300), seed=3),   # padding, n_rep 3
+    wl(1, 257, 4, 4, 128, 100, seed=4),            # d = 128
+    wl(1, 400, 2, 1, 128, 400, seed=5),            # d = 128, dense
+])
+def test_backward_matches_oracle(dma, case):
+    run_case(dma, case)

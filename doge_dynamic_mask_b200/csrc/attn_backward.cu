@@ -62,9 +62,11 @@ struct BwdCfg {
   static constexpr int kMetaBytes = 3 * kKeyTile * 4;
   static constexpr int kOffBar = kOffMeta + kStages * kMetaBytes;
   static constexpr int kSmemBytes = kOffBar + 128 + 1024;
-  // TMEM: S / dV_t at 0, dP / dK_t at 128 (dK_t is D + 16 wide), dQ after it
+  // TMEM: S / dV_t at 0, dP / dK_t at 128 (dK_t is D + 64 wide: Q's columns
+  // and the whole ones slab, so the MN-major B operand is made of full
+  // 64-column swizzle atoms), dQ after it
   static constexpr uint32_t kColDK = 128;
-  static constexpr uint32_t kColDQ = 128 + (D + 16 > 128 ? D + 16 : 128);
+  static constexpr uint32_t kColDQ = 128 + (D + 64 > 128 ? D + 64 : 128);
   static_assert(kColDQ + D <= 512, "TMEM budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
@@ -111,9 +113,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int nrows = min(kRowTile, L - r0);
   const int row = tid;
   const bool row_valid = row < nrows;
-  const int2 cnt = plan.counts[tile];
-  const int n_total = cnt.y;
-  const int n_kt = (n_total + kKeyTile - 1) / kKeyTile;
   const int base_row = b * L;
 
   unsigned char* sQ = smem + C::kOffQ;
@@ -149,7 +148,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  // everything above overlaps the previous kernel; the key lists and their
+  // counts come from it (the selector)
   pdl_wait();
+  const int2 cnt = plan.counts[tile];
+  const int n_total = cnt.y;
+  const int n_kt = (n_total + kKeyTile - 1) / kKeyTile;
 
   // D_r = dO_r . O_r (float32, from the rows in global memory)
   float Dr = 0.0f;
@@ -231,7 +235,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t idesc_s = make_idesc_bf16(128, 128, false, false);          // S, dP
   const uint32_t idesc_dq = make_idesc_bf16(128, D, false, true);            // dS (K-major) x K (MN-major)
   const uint32_t idesc_dv = make_idesc_bf16(128, D, true, true);             // P^T (MN-major) x dO (MN-major)
-  const uint32_t idesc_dk = make_idesc_bf16(128, D + 16, true, true);        // dS^T x [Q | 1]
+  const uint32_t idesc_dk = make_idesc_bf16(128, D + 64, true, true);        // dS^T x [Q | 1]
   const uint32_t q_lo = desc_lo(smem_u32(sQ), 16), do_lo = desc_lo(smem_u32(sDO), 16);
   const uint32_t qmn_lo = desc_lo(smem_u32(sQ), C::kSlabBytes);              // [Q | 1] as an MN-major B
   const uint32_t domn_lo = desc_lo(smem_u32(sDO), C::kSlabBytes);

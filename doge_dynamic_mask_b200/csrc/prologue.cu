@@ -18,8 +18,10 @@
 // cosines and sines kept in shared memory; then each group of d/8 lanes owns
 // one head row as sixteen-byte vectors (eight bf16 channels per lane): the
 // mean square is a group shuffle reduction, and channel i's rotation partner
-// i + d/2 sits in the lane d/16 positions away, one shuffle.  Arithmetic is
-// float32 with one rounding to bf16 at the end; V rows are copied bit for bit.
+// i + d/2 sits in the lane d/16 positions away, one shuffle.  Each lane keeps
+// four row pieces in flight (the first four are requested before the angles
+// are formed, and each piece's successor as soon as it is taken).  Arithmetic
+// is float32 with one rounding to bf16 at the end; V rows are copied bit for bit.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -38,6 +40,12 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float* f) {
   }
 }
 
+// One row-group step: this lane's 16-byte piece of head row r (q, k or v).
+struct RowPiece {
+  uint4 u;
+  int r;
+};
+
 template <int D>
 __global__ void __launch_bounds__(kPrologueThreads)
     prologue_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k, const uint4* __restrict__ v,
@@ -48,10 +56,32 @@ __global__ void __launch_bounds__(kPrologueThreads)
   constexpr int kLanesPerRow = D / 8;               // 16-byte vectors per head row
   constexpr int kRowsPerWarp = 32 / kLanesPerRow;
   constexpr int kHalf = kLanesPerRow / 2;           // lane distance of channel i's partner i + d/2
+  constexpr int kStride = (kPrologueThreads / 32) * kRowsPerWarp;   // rows per block step
+  constexpr int kBatch = 4;                         // block steps whose loads are in flight together
   __shared__ float s_cos[D / 2], s_sin[D / 2];
 
   const int token = blockIdx.x;                     // b * L + t
   const int b = token / L, t = token - b * L;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane % kLanesPerRow;              // this lane's 8 channels: [8 sub, 8 sub + 8)
+  const int rows = Hq + 2 * Hkv;                    // q heads, then k heads, then v heads
+  const size_t qrow0 = static_cast<size_t>(token) * Hq;
+  const size_t krow0 = static_cast<size_t>(token) * Hkv;
+  const int row_in_step = warp * kRowsPerWarp + lane / kLanesPerRow;
+
+  auto load = [&](int r) -> uint4 {
+    if (r >= rows) return make_uint4(0u, 0u, 0u, 0u);
+    if (r < Hq) return __ldcs(q + (qrow0 + r) * kLanesPerRow + sub);
+    if (r < Hq + Hkv) return __ldcs(k + (krow0 + (r - Hq)) * kLanesPerRow + sub);
+    return __ldcs(v + (krow0 + (r - Hq - Hkv)) * kLanesPerRow + sub);
+  };
+  // the first batch of rows is in flight while the angles are formed
+  RowPiece pc[kBatch];
+#pragma unroll
+  for (int it = 0; it < kBatch; ++it) {
+    pc[it].r = it * kStride + row_in_step;
+    pc[it].u = load(pc[it].r);
+  }
   const int pos = positions[b] + t;
   const bool in_cache = positions[b] >= 0 && pos < Lmax;
   if (threadIdx.x == 0 && !in_cache) raise_error(err, kDevErrBadPosition);
@@ -64,60 +94,57 @@ __global__ void __launch_bounds__(kPrologueThreads)
     s_sin[threadIdx.x] = static_cast<float>(sn);
   }
   __syncthreads();
+  const size_t crow0 = in_cache ? (static_cast<size_t>(b) * Lmax + pos) * Hkv : 0;
+  const bool low = sub < kHalf;                     // channels below d/2
+  const int i0 = 8 * (low ? sub : sub - kHalf);     // pair index of this lane's first channel
 
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int sub = lane % kLanesPerRow;              // this lane's 8 channels: [8 sub, 8 sub + 8)
-  const int rows = Hq + 2 * Hkv;                    // q heads, then k heads, then v heads
-  const size_t qrow0 = static_cast<size_t>(token) * Hq;
-  const size_t krow0 = static_cast<size_t>(token) * Hkv;
-  const size_t crow0 = (static_cast<size_t>(b) * Lmax + pos) * Hkv;
-  for (int base = warp * kRowsPerWarp; base < rows; base += (kPrologueThreads / 32) * kRowsPerWarp) {
-    const int r = base + lane / kLanesPerRow;
-    const bool live = r < rows;
-    const bool is_q = r < Hq, is_k = !is_q && r < Hq + Hkv;
-    uint4 u = make_uint4(0u, 0u, 0u, 0u);
-    if (live) {
-      if (is_q) u = q[(qrow0 + r) * kLanesPerRow + sub];
-      else if (is_k) u = k[(krow0 + (r - Hq)) * kLanesPerRow + sub];
-      else u = v[(krow0 + (r - Hq - Hkv)) * kLanesPerRow + sub];
-    }
-    if (live && !is_q && !is_k) {
-      if (in_cache) v_cache[(crow0 + (r - Hq - Hkv)) * kLanesPerRow + sub] = u;   // V: appended as is
-    }
-    // the shuffles below run on every lane of the warp (uniform trip count)
-    float x[8];
-    bf16x8_to_f32(u, x);
-    float ss = 0.0f;
+  for (int base = 0; base < rows; base += kBatch * kStride) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
-#pragma unroll
-    for (int o = kLanesPerRow / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
-    const float inv = 1.0f / sqrtf(ss * (1.0f / D) + eps);
-    const float* w = is_q ? q_w : k_w;
-    float y[8], yp[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) y[e] = (live && (is_q || is_k)) ? w[8 * sub + e] * (x[e] * inv) : 0.0f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) yp[e] = __shfl_xor_sync(0xFFFFFFFFu, y[e], kHalf);
-    if (live && (is_q || is_k)) {
-      const bool low = sub < kHalf;                 // channels below d/2
-      const int i0 = 8 * (low ? sub : sub - kHalf); // pair index of this lane's first channel
-      uint32_t pk[4];
-#pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        float o0, o1;
-        if (low) {
-          o0 = y[e] * s_cos[i0 + e] - yp[e] * s_sin[i0 + e];
-          o1 = y[e + 1] * s_cos[i0 + e + 1] - yp[e + 1] * s_sin[i0 + e + 1];
-        } else {
-          o0 = y[e] * s_cos[i0 + e] + yp[e] * s_sin[i0 + e];
-          o1 = y[e + 1] * s_cos[i0 + e + 1] + yp[e + 1] * s_sin[i0 + e + 1];
-        }
-        pk[e / 2] = pack_bf16x2(o0, o1);
+    for (int it = 0; it < kBatch; ++it) {
+      const int r = pc[it].r;
+      const uint4 u = pc[it].u;
+      // prefetch the same slot of the next batch
+      const int rn = r + kBatch * kStride;
+      if (base + kBatch * kStride < rows) pc[it].u = load(rn);
+      pc[it].r = rn;
+      const bool live = r < rows;
+      const bool is_q = r < Hq, is_k = !is_q && r < Hq + Hkv;
+      if (live && !is_q && !is_k) {
+        if (in_cache) v_cache[(crow0 + (r - Hq - Hkv)) * kLanesPerRow + sub] = u;   // V: appended as is
       }
-      const uint4 o = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      if (is_q) q_out[(qrow0 + r) * kLanesPerRow + sub] = o;
-      else if (in_cache) k_cache[(crow0 + (r - Hq)) * kLanesPerRow + sub] = o;
+      // the shuffles below run on every lane of the warp (uniform trip count)
+      float x[8];
+      bf16x8_to_f32(u, x);
+      float ss = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+#pragma unroll
+      for (int o = kLanesPerRow / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+      const float inv = 1.0f / sqrtf(ss * (1.0f / D) + eps);
+      const float* w = is_q ? q_w : k_w;
+      float y[8], yp[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] = (live && (is_q || is_k)) ? w[8 * sub + e] * (x[e] * inv) : 0.0f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) yp[e] = __shfl_xor_sync(0xFFFFFFFFu, y[e], kHalf);
+      if (live && (is_q || is_k)) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          float o0, o1;
+          if (low) {
+            o0 = y[e] * s_cos[i0 + e] - yp[e] * s_sin[i0 + e];
+            o1 = y[e + 1] * s_cos[i0 + e + 1] - yp[e + 1] * s_sin[i0 + e + 1];
+          } else {
+            o0 = y[e] * s_cos[i0 + e] + yp[e] * s_sin[i0 + e];
+            o1 = y[e + 1] * s_cos[i0 + e + 1] + yp[e + 1] * s_sin[i0 + e + 1];
+          }
+          pk[e / 2] = pack_bf16x2(o0, o1);
+        }
+        const uint4 o = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        if (is_q) __stcs(q_out + (qrow0 + r) * kLanesPerRow + sub, o);
+        else if (in_cache) k_cache[(crow0 + (r - Hq)) * kLanesPerRow + sub] = o;
+      }
     }
   }
 }

@@ -7,7 +7,11 @@ Bars (derived from the arithmetic): the kernels round P and dS to bf16 for
 the tensor core (relative error 2^-9 each, accumulated in float32 over up to
 a few thousand keys or rows with mixed signs) and round dq, dk, dv to bf16;
 every gradient G must satisfy
-  max |got - want| <= 2e-2 * max |want|   and   mean |got - want| <= 4e-3 * mean |want|.
+  max |got - want| <= 2e-2 * max |want|   and   mean |got - want| <= 4e-3 * mean |want|,
+except dA, a sum over every token of d_dt * dt * softplus(x) whose terms cancel
+almost completely (d_dt sums to zero over the keys, since each softmax row's
+dS does): its error is bounded by the same relative bar applied to the sum
+of the terms' magnitudes, |got - want| <= 2e-2 * sum |d_dt dt softplus(x)|.
 """
 import numpy as np
 import pytest
@@ -58,10 +62,17 @@ def run_case(dma, wl, dout_seed=1):
                                    torch.from_numpy(out).to(torch.bfloat16).cuda(), dout.cuda(),
                                    dt_in=torch.from_numpy(dt).cuda(), want_d_dt=True)
     torch.cuda.synchronize()
-    names = ("dq", "dk", "dv", "dW", "dA", "d_dt")
-    order = (0, 1, 2, 4, 5, 3)    # oracle returns dq, dk, dv, d_dt, dW, dA
-    for name, gi, wi in zip(names, range(6), order):
+    names = ("dq", "dk", "dv", "dW", "d_dt")
+    order = (0, 1, 2, 4, 3)    # oracle returns dq, dk, dv, d_dt, dW, dA
+    for name, gi, wi in zip(names, (0, 1, 2, 3, 5), order):
         assert_grad_close(got[gi], want[wi], name)
+    # dA: bar on the magnitude of its terms
+    B, L, Hkv, d = v.shape
+    x64 = v.reshape(B, L, Hkv * d) @ W
+    sp = oracle.softplus(x64)
+    terms = np.abs(want[3].transpose(0, 2, 1) * np.exp(A * sp) * sp).sum(axis=(0, 1))
+    err = np.abs(f64(got[4]) - want[5])
+    assert (err <= MAX_REL * terms).all(), (err, terms)
 
 
 def wl(B, L, Hq, Hkv, d, w, lens=None, seed=0):

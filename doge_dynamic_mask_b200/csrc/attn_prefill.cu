@@ -721,7 +721,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           mbar_arrive_warp(bars.s_free);   // S may be overwritten by the next Q K^T
         }
-        if (!((j + 1) * kKeyTile <= n_full || !row_valid)) {
+        if (plan.no_topk && !((j + 1) * kKeyTile <= n_full || !row_valid)) {
+          // every visible key kept: list entry e is key e, kept up to this
+          // row's causal limit and the last valid key
+          const int lim = min(r0 + row, x.n_total - 1) - j * kKeyTile;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c > lim) r[c] = __float_as_uint(-INFINITY);
+        } else if (!((j + 1) * kKeyTile <= n_full || !row_valid)) {
           // key tile not kept by every row: drop keys outside this row's interval
           const uint4* ms4 = reinterpret_cast<const uint4*>(sMeta + ms_slot * C::kMetaBytes);
 #pragma unroll

@@ -14,8 +14,9 @@
 // Design.  Memory-bound: every projected row is read once and written once.
 // One CTA per token: the d/2 angles of its position are formed in double
 // precision (a position of 10^5 times a frequency near 1 would lose about
-// 2^-7 rad of its angle in float32, the size of a bf16 rounding) and their
-// cosines and sines kept in shared memory; then each group of d/8 lanes owns
+// 2^-7 rad of its angle in float32, the size of a bf16 rounding) as turns,
+// reduced to their fractional part, and their cosines and sines taken in
+// float32 (sincospi) and kept in shared memory; then each group of d/8 lanes owns
 // one head row as sixteen-byte vectors (eight bf16 channels per lane): the
 // mean square is a group shuffle reduction, and channel i's rotation partner
 // i + d/2 sits in the lane d/16 positions away, one shuffle.  Each lane keeps
@@ -86,12 +87,16 @@ __global__ void __launch_bounds__(kPrologueThreads)
   const bool in_cache = positions[b] >= 0 && pos < Lmax;
   if (threadIdx.x == 0 && !in_cache) raise_error(err, kDevErrBadPosition);
   if (threadIdx.x < D / 2) {
-    // theta^(-2i/d) and the angle in double precision, then its cosine and sine
+    // the angle in turns, u = pos * theta^(-2i/d) / (2 pi), in double precision;
+    // its fractional part r in [-1/2, 1/2] (exact in float32 to 2^-25) gives
+    // cos and sin of 2 pi r = the angle modulo 2 pi, in float32
     const double inv_freq = exp(-2.0 * static_cast<double>(threadIdx.x) / D * log_theta);
-    double sn, cs;
-    sincos(static_cast<double>(pos) * inv_freq, &sn, &cs);
-    s_cos[threadIdx.x] = static_cast<float>(cs);
-    s_sin[threadIdx.x] = static_cast<float>(sn);
+    const double u = static_cast<double>(pos) * (inv_freq * 0.15915494309189535);   // 1 / (2 pi)
+    const float r = static_cast<float>(u - rint(u));
+    float sn, cs;
+    sincospif(2.0f * r, &sn, &cs);
+    s_cos[threadIdx.x] = cs;
+    s_sin[threadIdx.x] = sn;
   }
   __syncthreads();
   const size_t crow0 = in_cache ? (static_cast<size_t>(b) * Lmax + pos) * Hkv : 0;

@@ -64,7 +64,7 @@ namespace {
 // registers.  128 x kRegsControl + 256 x kRegsSoftmax must not exceed what the
 // block was launched with: the launcher checks it before every launch.
 constexpr int kThreads = 384;
-constexpr int kRegsControl = 72;
+constexpr int kRegsControl = 88;
 constexpr int kRegsSoftmax = 208;
 static_assert(kRegsControl % 8 == 0 && kRegsSoftmax % 8 == 0, "setmaxnreg takes multiples of 8");
 constexpr float kLog2e = 1.4426950408889634f;
@@ -405,7 +405,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* bias_t = plan.bias + x.tile * plan.cap;
       const uint32_t* span_t = plan.span + x.tile * plan.cap;
       const float* dt_row = plan.dt_src + (static_cast<size_t>(x.it.b) * Hkv + g) * L;
+      // One tile's list metadata for this lane's four entries: bias, row
+      // intervals, key indices and the tile's run start.  The loads of tile
+      // j + 1 are issued before waiting for tile j + 1's stage, so their
+      // latency overlaps that wait instead of following it.
+      struct TileMeta {
+        float bv[4];
+        uint4 sp;
+        int4 ix;
+        int kb0;
+      };
+      auto fetch_meta = [&](int j) {
+        TileMeta mt;
+        const int e = j * kKeyTile + lane * 4;
+        if (plan.no_topk) {
+          // list entry e is key e; padding past the last visible key has span 0
+          const int r0 = x.it.t * kRowTile, nrows = min(kRowTile, L - r0);
+          uint32_t spv[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int key = e + q;
+            const bool live = key < x.n_total;
+            mt.bv[q] = live ? dt_row[key] : 0.0f;
+            spv[q] = live ? static_cast<uint32_t>(key > r0 ? key - r0 : 0) | (static_cast<uint32_t>(nrows) << 16) : 0u;
+          }
+          mt.sp = make_uint4(spv[0], spv[1], spv[2], spv[3]);
+          mt.kb0 = j * kKeyTile;
+          mt.ix = make_int4(0, 0, 0, 0);
+        } else {
+          const float4 bi = *reinterpret_cast<const float4*>(bias_t + e);
+          mt.sp = *reinterpret_cast<const uint4*>(span_t + e);
+          mt.bv[0] = bi.x; mt.bv[1] = bi.y; mt.bv[2] = bi.z; mt.bv[3] = bi.w;
+          mt.kb0 = kbase_t[j];
+          mt.ix = *reinterpret_cast<const int4*>(idx_t + e);
+        }
+        return mt;
+      };
+      TileMeta nxt = fetch_meta(0);
       for (int j = 0; j < x.n_kt; ++j, ++gk) {
+        const TileMeta cur = nxt;
+        if (j + 1 < x.n_kt) nxt = fetch_meta(j + 1);
         const int s = gk % C::kStages;
         const int u = gk / C::kStages;
         const int ms_slot = gk % C::kMetaSlots;
@@ -418,29 +457,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           stop = true;
           break;
         }
-        const int e = j * kKeyTile + lane * 4;
-        const int kb0 = plan.no_topk ? j * kKeyTile : kbase_t[j];
+        const int kb0 = cur.kb0;
         {
-          float bv[4];
-          uint4 sp;
-          if (plan.no_topk) {
-            // list entry e is key e; padding past the last visible key has span 0
-            const int r0 = x.it.t * kRowTile, nrows = min(kRowTile, L - r0);
-            uint32_t spv[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int key = e + q;
-              const bool live = key < x.n_total;
-              bv[q] = live ? dt_row[key] : 0.0f;
-              spv[q] = live ? static_cast<uint32_t>(key > r0 ? key - r0 : 0) | (static_cast<uint32_t>(nrows) << 16)
-                            : 0u;
-            }
-            sp = make_uint4(spv[0], spv[1], spv[2], spv[3]);
-          } else {
-            const float4 bi = *reinterpret_cast<const float4*>(bias_t + e);
-            sp = *reinterpret_cast<const uint4*>(span_t + e);
-            bv[0] = bi.x; bv[1] = bi.y; bv[2] = bi.z; bv[3] = bi.w;
-          }
+          const float* bv = cur.bv;
+          const uint4 sp = cur.sp;
           *reinterpret_cast<uint4*>(sMeta + ms_slot * C::kMetaBytes + lane * 16) = sp;
 #pragma unroll
           for (int q = 0; q < 4; ++q)
@@ -449,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();   // the bias block is read by the tensor core
         int4 ix = make_int4(0, 0, 0, 0);
         if (kb0 < 0) {
-          ix = *reinterpret_cast<const int4*>(idx_t + e);
+          ix = cur.ix;
           ix.x = (base_row + ix.x) * Hkv + g;
           ix.y = (base_row + ix.y) * Hkv + g;
           ix.z = (base_row + ix.z) * Hkv + g;
@@ -492,7 +512,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int g = x.it.g, base_row = x.it.b * L;
       const int32_t* idx_t = plan.idx + x.tile * plan.cap;
       const int32_t* kbase_t = plan.kbase + x.tile * (plan.cap / kKeyTile);
+      // the next tile's run start and key indices are fetched one tile ahead
+      auto fetch_kb = [&](int j) { return plan.no_topk ? j * kKeyTile : kbase_t[j]; };
+      auto fetch_ix = [&](int j) {
+        return plan.no_topk ? make_int4(0, 0, 0, 0) : *reinterpret_cast<const int4*>(idx_t + j * kKeyTile + lane * 4);
+      };
+      int nkb = x.n_kt > 0 ? fetch_kb(0) : 0;
+      int4 nix = x.n_kt > 0 ? fetch_ix(0) : make_int4(0, 0, 0, 0);
       for (int j = 0; j < x.n_kt; ++j, ++gv) {
+        const int kb0 = nkb;
+        int4 ix = nix;
+        if (j + 1 < x.n_kt) {
+          nkb = fetch_kb(j + 1);
+          nix = fetch_ix(j + 1);
+        }
         const int s = gv % C::kStages;
         const int u = gv / C::kStages;
         if (gv >= C::kStages && !mbar_wait(bars.v_empty + s, (u - 1) & 1, err, kDevErrTimeoutBase + 14)) {
@@ -504,10 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           stop = true;
           break;
         }
-        const int kb0 = plan.no_topk ? j * kKeyTile : kbase_t[j];
-        int4 ix = make_int4(0, 0, 0, 0);
         if (kb0 < 0) {
-          ix = *reinterpret_cast<const int4*>(idx_t + j * kKeyTile + lane * 4);
           ix.x = (base_row + ix.x) * Hkv + g;
           ix.y = (base_row + ix.y) * Hkv + g;
           ix.z = (base_row + ix.z) * Hkv + g;

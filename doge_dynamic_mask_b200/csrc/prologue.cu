@@ -19,10 +19,13 @@
 // float32 (sincospi) and kept in shared memory; then each group of d/8 lanes owns
 // one head row as sixteen-byte vectors (eight bf16 channels per lane): the
 // mean square is a group shuffle reduction, and channel i's rotation partner
-// i + d/2 sits in the lane d/16 positions away, one shuffle.  Each lane keeps
-// four row pieces in flight (the first four are requested before the angles
-// are formed, and each piece's successor as soon as it is taken).  Arithmetic
-// is float32 with one rounding to bf16 at the end; V rows are copied bit for bit.
+// i + d/2 sits in the lane d/16 positions away, one shuffle.  A lane's
+// channels are the same for every row it handles, so its norm weights,
+// cosines and sines live in registers (shared memory and L1 then carry only
+// the rows).  Each lane keeps two row pieces in flight (the first two are
+// requested before the angles are formed, and each piece's successor as soon
+// as it is taken).  Arithmetic is float32 with one rounding to bf16 at the
+// end; V rows are copied bit for bit.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -58,7 +61,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
   constexpr int kRowsPerWarp = 32 / kLanesPerRow;
   constexpr int kHalf = kLanesPerRow / 2;           // lane distance of channel i's partner i + d/2
   constexpr int kStride = (kPrologueThreads / 32) * kRowsPerWarp;   // rows per block step
-  constexpr int kBatch = 4;                         // block steps whose loads are in flight together
+  constexpr int kBatch = 2;                         // block steps whose loads are in flight together
   __shared__ float s_cos[D / 2], s_sin[D / 2];
 
   const int token = blockIdx.x;                     // b * L + t
@@ -102,6 +105,16 @@ __global__ void __launch_bounds__(kPrologueThreads)
   const size_t crow0 = in_cache ? (static_cast<size_t>(b) * Lmax + pos) * Hkv : 0;
   const bool low = sub < kHalf;                     // channels below d/2
   const int i0 = 8 * (low ? sub : sub - kHalf);     // pair index of this lane's first channel
+  // this lane's channels never change: its norm weights, cosines and sines
+  // are held in registers for every row it handles
+  float wq[8], wk[8], cs8[8], sn8[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    wq[e] = q_w[8 * sub + e];
+    wk[e] = k_w[8 * sub + e];
+    cs8[e] = s_cos[i0 + e];
+    sn8[e] = low ? -s_sin[i0 + e] : s_sin[i0 + e];   // the low half subtracts its partner's share
+  }
 
   for (int base = 0; base < rows; base += kBatch * kStride) {
 #pragma unroll
@@ -126,24 +139,17 @@ __global__ void __launch_bounds__(kPrologueThreads)
 #pragma unroll
       for (int o = kLanesPerRow / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
       const float inv = 1.0f / sqrtf(ss * (1.0f / D) + eps);
-      const float* w = is_q ? q_w : k_w;
       float y[8], yp[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) y[e] = (live && (is_q || is_k)) ? w[8 * sub + e] * (x[e] * inv) : 0.0f;
+      for (int e = 0; e < 8; ++e) y[e] = (live && (is_q || is_k)) ? (is_q ? wq[e] : wk[e]) * (x[e] * inv) : 0.0f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) yp[e] = __shfl_xor_sync(0xFFFFFFFFu, y[e], kHalf);
       if (live && (is_q || is_k)) {
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 8; e += 2) {
-          float o0, o1;
-          if (low) {
-            o0 = y[e] * s_cos[i0 + e] - yp[e] * s_sin[i0 + e];
-            o1 = y[e + 1] * s_cos[i0 + e + 1] - yp[e + 1] * s_sin[i0 + e + 1];
-          } else {
-            o0 = y[e] * s_cos[i0 + e] + yp[e] * s_sin[i0 + e];
-            o1 = y[e + 1] * s_cos[i0 + e + 1] + yp[e + 1] * s_sin[i0 + e + 1];
-          }
+          const float o0 = fmaf(yp[e], sn8[e], y[e] * cs8[e]);
+          const float o1 = fmaf(yp[e + 1], sn8[e + 1], y[e + 1] * cs8[e + 1]);
           pk[e / 2] = pack_bf16x2(o0, o1);
         }
         const uint4 o = make_uint4(pk[0], pk[1], pk[2], pk[3]);

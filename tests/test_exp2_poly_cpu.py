@@ -72,3 +72,20 @@ def test_no_sign_or_inf_for_any_input():
     assert np.isfinite(p).all() and (p >= 0).all()
     below = x <= -126.0
     assert p[below].max() <= np.exp2(-125.0)   # effectively zero next to the row maximum's weight 1
+
+
+def test_cubic_is_the_minimax_fit_of_the_relative_error():
+    """The cubic is the best uniform (minimax) fit of 2^f's relative error on
+    [-1/2, 1/2]: by the Chebyshev alternation theorem a cubic is that fit
+    exactly when its error reaches its maximum magnitude at five points with
+    alternating signs (the two ends and three interior extrema)."""
+    _, _, (c0, c1, c2, c3) = _constants()
+    f = np.linspace(-0.5, 0.5, 400001)
+    rel = (float(c0) + f * (float(c1) + f * (float(c2) + f * float(c3)))) / np.exp2(f) - 1.0
+    inner = np.nonzero(np.diff(np.sign(np.diff(rel))))[0] + 1
+    pts = np.concatenate([[0], inner, [len(f) - 1]])
+    assert len(pts) == 5
+    vals = rel[pts]
+    assert (np.sign(vals[1:]) != np.sign(vals[:-1])).all()             # alternating signs
+    assert np.abs(vals).min() >= 0.999 * np.abs(rel).max()              # equal magnitude
+    assert np.abs(rel).max() < 7.5e-5

@@ -10,26 +10,30 @@
 // Prefill (one CTA per (batch, kv head, run of consecutive 128-row tiles)).
 // dt does not depend on the query, so the row threshold tau_i (the composite
 // key of row i's worst kept key) never decreases along the rows: each key is
-// kept on one contiguous interval of rows, and the union of the kept sets of a
-// row tile is the w keys kept at its first row plus at most 127 newer keys.
-// For each tile of its run the CTA
-//   1. finds tau at the tile's first row: by radix selection over the keys
-//      that row sees (the run's first tile), or from the previous tile's
-//      last-row kept set plus at most one new key (every later tile),
-//   2. collects the union U (keys <= the tile's last visible row whose key is
-//      >= that tau) in index order: from the prefix in global memory, or from
-//      the previous tile's union and the tile's own new keys,
-//   3. takes the 128 smallest keys of U, in which every later row's tau lies,
-//      and resolves tau_i for each row of the tile,
-//   4. gives each key of U its row interval [lo, hi) inside the tile and writes
-//      the list: keys kept by every row first, then the rest (index order in
-//      each class), each with its dt bias and interval.
+// kept on one contiguous interval of rows, and the union U of the kept sets of
+// a row tile is the w keys kept at its first row plus at most 127 newer keys.
+// The CTA keeps U sorted by key.  For each tile of its run it
+//   1. has K, the kept set at the tile's first row, sorted: for the run's first
+//      tile by selecting the w-th largest key over the prefix (radix
+//      histogram, then one collection pass) and sorting the w keys in shared
+//      memory; for every later tile it is the previous tile's K(q), the first
+//      w keys of the previous union, less at most its smallest key,
+//   2. merges the tile's new keys that pass the first-row threshold into K,
+//      giving U,
+//   3. resolves tau_i for each row among the 128 smallest keys of U (the tail,
+//      in which every row's tau lies),
+//   4. gives each key its row interval [lo, hi) inside the tile (a key above
+//      the tail is never evicted in the tile) and writes the list: keys kept
+//      by every row first, then the rest, each with its dt bias and interval
+//      (the order inside a class carries no meaning).
 // Tiles whose rows see at most w keys (and every tile when Lk <= w) keep
-// every visible key and skip the selection.
+// every visible key and skip the selection; their lists are in index order.
 //
 // Decode (one CTA per (batch, kv head)): the single query at len_b - 1 keeps
 // the w best of its len_b keys; radix-select the w-th key, then compact the
 // kept keys in index order.
+#include <algorithm>
+
 #include "select_common.cuh"
 
 namespace dma {
@@ -40,12 +44,34 @@ struct SelectSmem {
   uint64_t cand[kCandCap];
   uint32_t red[64];
   uint64_t vars[8];
-  uint64_t tau_s[kRowTile];
-  uint64_t bot[kRowTile];
-  uint64_t bot_raw[kRowTile];
-  int misc[8];
-  // followed by two unions U[ucap] (uint64) in dynamic shared memory
 };
+
+// Prefill selector state; the candidate buffer of the prefix selection shares
+// the dynamic region with the two key buffers (it is dead before they are
+// written).
+struct PrefillSelSmem {
+  uint32_t hist[kBins];
+  uint32_t red[64];
+  uint64_t vars[8];
+  uint64_t newk[kRowTile];      // the tile's new keys that pass tau0 (0: none), then sorted
+  uint64_t news[kRowTile];      // the passing new keys, descending
+  int32_t ins[kRowTile];        // keys of K above each of them
+  uint64_t tau_s[kRowTile];     // tau of each row of the tile
+  int32_t pos_s[kRowTile];      // ascending tail position of each row's tau (-1: the row keeps every visible key)
+  int16_t rowpos[kRowTile];     // tail position of the union key whose index is r0 + offset, or -1
+  uint32_t newmask[kRowTile / 32];    // row offsets j - r0 of the union's keys newer than the first row
+  uint32_t oldmask[kRowTile / 32];    // tail positions of keys every row sees
+  uint32_t wor[kRowTile / 32][kRowTile / 32];   // per-warp OR of the rows' new-key tail bits
+  uint8_t hi_tail[kRowTile];    // first row whose tau lies above the tail key
+  uint32_t cnt[2][kRowTile / 32];    // per-warp counts of the tail's evicted and dead keys
+  uint32_t tot[4];
+  uint64_t nextk;               // composite key of the next tile's first row
+  // followed in dynamic shared memory by two key buffers of ucap keys
+};
+
+// prefill selector CTA: threads, and CTAs resident per SM (64 registers a thread)
+constexpr int kSelPrefillThreads = 512;
+constexpr int kSelPrefillMinBlocks = 2;
 
 // at most this many consecutive row tiles per prefill-selector CTA (see
 // select_prefill_kernel); the launcher picks fewer when the grid would not
@@ -61,48 +87,396 @@ __device__ __forceinline__ int clamp_len(const int32_t* lengths, int b, int L, u
   return len;
 }
 
-// Minimum of the keys of U[0, n) above `floor` (~0 when there is none).
-__device__ __forceinline__ uint64_t block_min_above(const uint64_t* U, int n, uint64_t floor, uint64_t* scratch) {
-  uint64_t m = ~0ull;
-  for (int e = threadIdx.x; e < n; e += blockDim.x) {
-    const uint64_t k = U[e];
-    if (k > floor && k < m) m = k;
-  }
+// Bit position of the k-th (1-based) set bit of b; 1 <= k <= popc(b).
+__device__ __forceinline__ int nth_set_bit(uint32_t b, int k) {
+  int pos = 0;
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    const uint64_t x = __shfl_xor_sync(0xFFFFFFFFu, m, o);
-    m = x < m ? x : m;
+  for (int width = 16; width >= 1; width >>= 1) {
+    const int c = __popc(b & ((1u << width) - 1u));
+    if (c < k) {
+      k -= c;
+      b >>= width;
+      pos += width;
+    }
   }
-  const int warp = threadIdx.x >> 5;
+  return pos;
+}
+
+// Number of set bits at offsets [0, lim] of a 128-bit mask (0 when lim < 0).
+__device__ __forceinline__ int popc_upto(const uint32_t* m, int lim) {
+  int c = 0;
+#pragma unroll
+  for (int wd = 0; wd < 4; ++wd) {
+    const int top = lim - 32 * wd;
+    if (top >= 31) c += __popc(m[wd]);
+    else if (top >= 0) c += __popc(m[wd] & ((2u << top) - 1u));
+  }
+  return c;
+}
+
+__device__ __forceinline__ uint64_t shfl_xor64(uint64_t v, int m) {
+  const uint32_t lo = __shfl_xor_sync(0xFFFFFFFFu, static_cast<uint32_t>(v), m);
+  const uint32_t hi = __shfl_xor_sync(0xFFFFFFFFu, static_cast<uint32_t>(v >> 32), m);
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+// Number of entries of the descending array a[0, n) greater than v (v not in a).
+__device__ __forceinline__ int count_greater(const uint64_t* a, int n, uint64_t v) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (a[mid] > v) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+// Bitonic compare-exchange stages with partner distance j <= 16 for block size k,
+// on one key per lane; e is the key's position in the whole sequence (its
+// bits pick the direction: the lower position keeps the larger key where
+// (e & k) == 0, so the final sequence is descending).
+__device__ __forceinline__ uint64_t bitonic_warp_stages(uint64_t v, int e, int k) {
+#pragma unroll
+  for (int j = 16; j > 0; j >>= 1) {
+    if (j < k) {
+      const uint64_t o = shfl_xor64(v, j);
+      const bool keep_max = ((e & j) == 0) == ((e & k) == 0);
+      v = keep_max ? (o > v ? o : v) : (o < v ? o : v);
+    }
+  }
+  return v;
+}
+
+// Sorts the n distinct keys (all > 0) of a[0, n) in descending order, in
+// place; a must have room for pow2 = max(32, next power of two >= n) keys
+// (the rest is padded with 0, which sorts last).  Stages with partner distance
+// up to 16 run on registers (one key per lane, shuffles), the longer ones as
+// pair passes over shared memory.  Every thread must call it.
+__device__ void block_bitonic_desc(uint64_t* a, int n) {
+  int pow2 = 32;
+  while (pow2 < n) pow2 <<= 1;
+  for (int e = n + threadIdx.x; e < pow2; e += blockDim.x) a[e] = 0ull;
   __syncthreads();
-  if ((threadIdx.x & 31) == 0) scratch[warp] = m;
+  const int lane = static_cast<int>(lane_id()), warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int base = warp * 32; base < pow2; base += nw * 32) {   // blocks of 2 .. 32
+    const int e = base + lane;
+    uint64_t v = a[e];
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) v = bitonic_warp_stages(v, e, k);
+    a[e] = v;
+  }
   __syncthreads();
-  uint64_t r = ~0ull;
-  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) r = scratch[w] < r ? scratch[w] : r;
+  for (int k = 64; k <= pow2; k <<= 1) {
+    for (int j = k >> 1; j >= 32; j >>= 1) {
+      for (int i = threadIdx.x; i < (pow2 >> 1); i += blockDim.x) {
+        const int x = ((i & ~(j - 1)) << 1) | (i & (j - 1)), y = x + j;
+        const uint64_t u = a[x], v = a[y];
+        const uint64_t big = u > v ? u : v, small = u > v ? v : u;
+        const bool desc = (x & k) == 0;
+        a[x] = desc ? big : small;
+        a[y] = desc ? small : big;
+      }
+      __syncthreads();
+    }
+    for (int base = warp * 32; base < pow2; base += nw * 32) {
+      const int e = base + lane;
+      a[e] = bitonic_warp_stages(a[e], e, k);
+    }
+    __syncthreads();
+  }
+}
+
+// Sorts the n distinct keys of a[0, n) in descending order into a, with tmp
+// (n keys) as scratch and hist (kBins words): keys are bucketed by the 11
+// bits below the highest bit in which they differ, each bucket taking the
+// range of positions its rank among the buckets gives, and each key is then
+// placed by its rank inside its bucket.  Returns false, with a unchanged, when
+// a bucket holds more than 32 keys (the caller sorts another way).  Every
+// thread must call it.
+__device__ bool block_bucket_sort_desc(uint64_t* a, uint64_t* tmp, int n, uint32_t* hist, uint32_t* red) {
+  uint64_t vor = 0ull, vand = ~0ull;
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    vor |= a[e];
+    vand &= a[e];
+  }
+  uint64_t O, A;
+  block_or_and64(vor, vand, red, O, A);
+  const uint64_t vary = O ^ A;
+  if (vary == 0ull) return true;   // at most one key
+  const int hb = 63 - __clzll(static_cast<long long>(vary));
+  const int sh = hb >= 10 ? hb - 10 : 0;
+  auto digit = [&](uint64_t k) { return static_cast<int>((k >> sh) & static_cast<uint64_t>(kBins - 1)); };
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0u;
   __syncthreads();
-  return r;
+  for (int e = threadIdx.x; e < n; e += blockDim.x) atomicAdd(&hist[digit(a[e])], 1u);
+  __syncthreads();
+  // bucket starts from the top bucket down: off[d] = keys in buckets above d
+  const int per = (kBins + blockDim.x - 1) / blockDim.x;
+  const int top = kBins - static_cast<int>(threadIdx.x) * per;   // this thread's buckets [top - per, top)
+  uint32_t local = 0, biggest = 0;
+  for (int d = top - 1; d >= top - per && d >= 0; --d) {
+    const uint32_t h = hist[d];
+    local += h;
+    biggest = h > biggest ? h : biggest;
+  }
+  if (__syncthreads_or(biggest > 32u)) return false;
+  uint32_t total;
+  uint32_t run = block_exclusive_scan(local, red, &total);
+  for (int d = top - 1; d >= top - per && d >= 0; --d) {
+    const uint32_t h = hist[d];
+    hist[d] = run;
+    run += h;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    const uint64_t k = a[e];
+    tmp[atomicAdd(&hist[digit(k)], 1u)] = k;
+  }
+  __syncthreads();
+  // hist[d] is now the end of bucket d, and bucket d starts where bucket d + 1 ends
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    const uint64_t k = tmp[e];
+    const int d = digit(k);
+    const int st = d + 1 < kBins ? static_cast<int>(hist[d + 1]) : 0, en = static_cast<int>(hist[d]);
+    int r = 0;
+    for (int f = st; f < en; ++f) r += tmp[f] > k;
+    a[st + r] = k;
+  }
+  __syncthreads();
+  return true;
+}
+
+// Appends, in any order, the composite keys of positions [0, n) of a dt row
+// that are >= tau to X (at most cap); returns their number.  Each warp
+// reserves room for sixteen keys per lane with one shared-memory atomic.
+// Every thread must call it.
+__device__ int row_collect_ge(const uint32_t* __restrict__ bits, int n, uint64_t tau, uint64_t* X, int cap,
+                              unsigned long long* counter) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const uint32_t lane = lane_id(), lt = lanemask_lt();
+  if (tid == 0) *counter = 0ull;
+  __syncthreads();
+  const bool vec = (reinterpret_cast<uintptr_t>(bits) & 15u) == 0;
+  const int nq = vec ? (n >> 2) : 0;
+  const uint4* qv = reinterpret_cast<const uint4*>(bits);
+  for (int r0 = 0; r0 < nq; r0 += 4 * nt) {   // same trip count in every thread
+    uint32_t v[16];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = r0 + u * nt + tid;
+      const uint4 x = i < nq ? __ldg(qv + i) : make_uint4(0u, 0u, 0u, 0u);
+      v[4 * u] = x.x;
+      v[4 * u + 1] = x.y;
+      v[4 * u + 2] = x.z;
+      v[4 * u + 3] = x.w;
+    }
+    uint32_t vote[16];
+    uint32_t total = 0;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const int i = r0 + (c >> 2) * nt + tid;
+      const bool m = i < nq && composite_key(v[c], static_cast<uint32_t>(4 * i + (c & 3))) >= tau;
+      vote[c] = __ballot_sync(0xFFFFFFFFu, m);
+      total += __popc(vote[c]);
+    }
+    uint32_t base = 0;
+    if (lane == 0 && total) base = static_cast<uint32_t>(atomicAdd(counter, static_cast<unsigned long long>(total)));
+    base = __shfl_sync(0xFFFFFFFFu, base, 0);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const int i = r0 + (c >> 2) * nt + tid;
+      if ((vote[c] >> lane) & 1u) {
+        const uint32_t pos = base + __popc(vote[c] & lt);
+        if (pos < static_cast<uint32_t>(cap)) X[pos] = composite_key(v[c], static_cast<uint32_t>(4 * i + (c & 3)));
+      }
+      base += __popc(vote[c]);
+    }
+  }
+  for (int j0 = nq << 2; j0 < n; j0 += nt) {   // the rest of the row (or a row not 16-byte aligned)
+    const int j = j0 + tid;
+    uint64_t key = 0ull;
+    const bool m = j < n && (key = composite_key(__ldg(bits + j), static_cast<uint32_t>(j))) >= tau;
+    const uint32_t vote = __ballot_sync(0xFFFFFFFFu, m);
+    uint32_t base = 0;
+    if (lane == 0 && vote) base = static_cast<uint32_t>(atomicAdd(counter, static_cast<unsigned long long>(__popc(vote))));
+    base = __shfl_sync(0xFFFFFFFFu, base, 0);
+    if (m) {
+      const uint32_t pos = base + __popc(vote & lt);
+      if (pos < static_cast<uint32_t>(cap)) X[pos] = key;
+    }
+  }
+  __syncthreads();
+  const int r = static_cast<int>(*counter);
+  __syncthreads();
+  return r < cap ? r : cap;
+}
+
+// Collects the composite keys of positions [0, n) of a dt row by class:
+// cls(v) == 1 appends the key at the front of out (positions 0, 1, ...),
+// cls(v) == 2 at the back (positions cap - 1, cap - 2, ...), any order within
+// a class; counters[0] and counters[1] end as the two counts.  Each warp
+// reserves room for sixteen keys per lane with one shared-memory atomic per
+// class.  Every thread must call it.
+template <class Cls>
+__device__ void row_collect2(const uint32_t* __restrict__ bits, int n, Cls cls, uint64_t* out, int cap,
+                             unsigned long long* counters) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const uint32_t lane = lane_id(), lt = lanemask_lt();
+  if (tid < 2) counters[tid] = 0ull;
+  __syncthreads();
+  auto place = [&](uint32_t vf, uint32_t vb, uint32_t& bf, uint32_t& bb, uint64_t key) {
+    if ((vf >> lane) & 1u) {
+      const uint32_t pos = bf + __popc(vf & lt);
+      if (pos < static_cast<uint32_t>(cap)) out[pos] = key;
+    } else if ((vb >> lane) & 1u) {
+      const uint32_t pos = bb + __popc(vb & lt);
+      if (pos < static_cast<uint32_t>(cap)) out[cap - 1 - pos] = key;
+    }
+    bf += __popc(vf);
+    bb += __popc(vb);
+  };
+  const bool vec = (reinterpret_cast<uintptr_t>(bits) & 15u) == 0;
+  const int nq = vec ? (n >> 2) : 0;
+  const uint4* qv = reinterpret_cast<const uint4*>(bits);
+  for (int r0 = 0; r0 < nq; r0 += 4 * nt) {   // same trip count in every thread
+    uint32_t v[16];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = r0 + u * nt + tid;
+      const uint4 x = i < nq ? __ldg(qv + i) : make_uint4(0u, 0u, 0u, 0u);
+      v[4 * u] = x.x;
+      v[4 * u + 1] = x.y;
+      v[4 * u + 2] = x.z;
+      v[4 * u + 3] = x.w;
+    }
+    uint32_t vf[16], vb[16];
+    uint32_t tf = 0, tb = 0;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const int i = r0 + (c >> 2) * nt + tid;
+      const int k = i < nq ? cls(v[c]) : 0;
+      vf[c] = __ballot_sync(0xFFFFFFFFu, k == 1);
+      vb[c] = __ballot_sync(0xFFFFFFFFu, k == 2);
+      tf += __popc(vf[c]);
+      tb += __popc(vb[c]);
+    }
+    uint32_t bf = 0, bb = 0;
+    if (lane == 0) {
+      if (tf) bf = static_cast<uint32_t>(atomicAdd(counters, static_cast<unsigned long long>(tf)));
+      if (tb) bb = static_cast<uint32_t>(atomicAdd(counters + 1, static_cast<unsigned long long>(tb)));
+    }
+    bf = __shfl_sync(0xFFFFFFFFu, bf, 0);
+    bb = __shfl_sync(0xFFFFFFFFu, bb, 0);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const int i = r0 + (c >> 2) * nt + tid;
+      place(vf[c], vb[c], bf, bb, composite_key(v[c], static_cast<uint32_t>(4 * i + (c & 3))));
+    }
+  }
+  for (int j0 = nq << 2; j0 < n; j0 += nt) {   // the rest of the row (or a row not 16-byte aligned)
+    const int j = j0 + tid;
+    const uint32_t b = j < n ? __ldg(bits + j) : 0u;
+    const int k = j < n ? cls(b) : 0;
+    const uint32_t vf = __ballot_sync(0xFFFFFFFFu, k == 1), vb = __ballot_sync(0xFFFFFFFFu, k == 2);
+    uint32_t bf = 0, bb = 0;
+    if (lane == 0) {
+      if (vf) bf = static_cast<uint32_t>(atomicAdd(counters, static_cast<unsigned long long>(__popc(vf))));
+      if (vb) bb = static_cast<uint32_t>(atomicAdd(counters + 1, static_cast<unsigned long long>(__popc(vb))));
+    }
+    bf = __shfl_sync(0xFFFFFFFFu, bf, 0);
+    bb = __shfl_sync(0xFFFFFFFFu, bb, 0);
+    place(vf, vb, bf, bb, composite_key(b, static_cast<uint32_t>(j)));
+  }
+  __syncthreads();
+}
+
+// K(p) for n > w: the w largest composite keys among positions [0, n) of a dt
+// row, in any order, into out[0, w); *tau gets the w-th largest.  Three passes
+// over the row: which dt bits vary (OR / AND), an 11-bit histogram of the
+// highest varying bits, and one collection of every key in or above the bin
+// B holding the w-th largest (keys above B from the front of out, keys in B
+// from its back); tau is then selected among B's keys in shared memory and
+// B's keys at or above it join the front.  Returns false, with nothing
+// written, when B's keys would not fit beside the w (the caller selects and
+// collects another way).  Every thread must call it.
+__device__ bool prefix_topw(const uint32_t* __restrict__ bits, int n, int w, uint64_t* out, int cap, SelScratch sc,
+                            unsigned long long* counters, uint64_t* tau) {
+  uint32_t vor = 0u, vand = ~0u;
+  row_for_each(bits, n, [&](uint32_t v, int, bool ok) {
+    if (ok) {
+      vor |= v;
+      vand &= v;
+    }
+  });
+  uint64_t O, A;
+  block_or_and64(vor, vand, sc.red, O, A);
+  const uint32_t vary = static_cast<uint32_t>(O ^ A) ;
+  if (vary == 0u) {   // one dt value: the lowest w indices rank highest
+    for (int e = threadIdx.x; e < w; e += blockDim.x) out[e] = composite_key(static_cast<uint32_t>(A), e);
+    *tau = composite_key(static_cast<uint32_t>(A), static_cast<uint32_t>(w - 1));
+    __syncthreads();
+    return true;
+  }
+  const int hb = 31 - __clz(vary);
+  const int sh = hb >= 10 ? hb - 10 : 0;
+  const int nb = 1 << (hb - sh + 1);
+  const uint32_t mask = static_cast<uint32_t>(nb - 1);
+  for (int i = threadIdx.x; i < nb; i += blockDim.x) sc.hist[i] = 0u;
+  __syncthreads();
+  row_for_each(bits, n, [&](uint32_t v, int, bool ok) {
+    if (ok) atomicAdd(&sc.hist[(v >> sh) & mask], 1u);
+  });
+  __syncthreads();
+  uint32_t k_in_bin, cnt_b;
+  const uint32_t B = find_bin_from_top(sc.hist, nb, static_cast<uint32_t>(w), sc.red, sc.vars, &k_in_bin, &cnt_b);
+  const int above = w - static_cast<int>(k_in_bin);
+  if (w + static_cast<int>(cnt_b) > cap) return false;
+  row_collect2(
+      bits, n, [&](uint32_t v) { const uint32_t d = (v >> sh) & mask; return d > B ? 1 : (d == B ? 2 : 0); }, out, cap,
+      counters);
+  // tau: the k_in_bin-th largest of B's keys, out[cap - cnt_b, cap)
+  uint64_t* binb = out + (cap - static_cast<int>(cnt_b));
+  const uint64_t t = select_kth_smem(binb, static_cast<int>(cnt_b), k_in_bin, sc);
+  if (threadIdx.x == 0) counters[0] = 0ull;
+  __syncthreads();
+  for (int e = threadIdx.x; e < static_cast<int>(cnt_b); e += blockDim.x) {
+    const uint64_t k = binb[e];
+    if (k >= t) out[above + static_cast<int>(atomicAdd(counters, 1ull))] = k;
+  }
+  __syncthreads();
+  *tau = t;
+  return true;
 }
 
 // One CTA per (batch, kv head, run of tpc consecutive row tiles).
-// The first tile of the run whose rows need the top-k does the full
-// selection over its prefix.  Each following tile is derived from the one
-// before, in shared memory: the kept set at the previous tile's last visible
-// row K(q') (the w keys of the previous union U' at or above that row's tau)
-// plus at most one new key (the tile's first row, when it is a valid row)
-// gives the tile's first-row threshold as the w-th largest of w+1 keys, and
-// the new union is U' filtered by that threshold followed by the tile's own
-// new keys (q', q] that pass it.
-__global__ void __launch_bounds__(kSelThreads, 2) select_prefill_kernel(const float* __restrict__ dt,
+//
+// The CTA keeps the union U of a tile (the keys any of its rows keeps) sorted
+// by composite key, descending.  All of U is visible at the tile's last row q,
+// so the kept set there, K(q), is U's first w keys: it carries to the next
+// tile as is.  The next tile's first-row threshold tau0 is the w-th largest of
+// K(q) and the key of its first row p (tau_last = U[w-1], second smallest
+// U[w-2]); its union is K(q) without the keys below tau0 (at most the last)
+// merged with its new keys (q, q'] at or above tau0, sorted.  The first tile of
+// a run selects tau0 over its prefix, collects K(p) and sorts it.
+//
+// Every row's tau lies among the 128 smallest keys of U (a row sees at most
+// |U| - w keys fewer than U holds), the tail of the sorted union: row i's tau
+// is its rank-th visible tail key in ascending order, rank = (visible keys of
+// U) - w + 1, with the tail keys every row sees and the prefix-OR over rows of
+// the new ones.  A key above the tail is never evicted inside the tile; a tail
+// key is kept up to the first row whose tau lies above it.  The list holds the
+// keys every row keeps, then the others, each class in U's (descending key)
+// order; consecutive lanes write consecutive entries.
+__global__ void __launch_bounds__(kSelPrefillThreads, kSelPrefillMinBlocks) select_prefill_kernel(const float* __restrict__ dt,
                                                                      const int32_t* __restrict__ lengths, int Hkv,
                                                                      int L, int w, int tpc, PrefillPlan plan,
                                                                      uint32_t* err) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  SelectSmem& sm = *reinterpret_cast<SelectSmem*>(smem_raw);
+  PrefillSelSmem& sm = *reinterpret_cast<PrefillSelSmem*>(smem_raw);
   pdl_wait();      // dt comes from the previous kernel
   pdl_trigger();   // the attention may be scheduled
   const int ucap = w + kRowTile;
-  uint64_t* Ubuf = reinterpret_cast<uint64_t*>(smem_raw + sizeof(SelectSmem));   // two unions of ucap keys
-  SelScratch sc{sm.hist, sm.cand, sm.red, sm.vars};
+  uint64_t* Ubuf = reinterpret_cast<uint64_t*>(smem_raw + sizeof(PrefillSelSmem));   // two buffers of ucap keys
+  SelScratch sc{sm.hist, Ubuf, sm.red, sm.vars};   // the candidate buffer is dead before Ubuf is written
 
   const int g = blockIdx.y, b = blockIdx.z;
   const int len = clamp_len(lengths, b, L, err);
@@ -110,13 +484,16 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_prefill_kernel(const fl
   const size_t bg = static_cast<size_t>(b) * Hkv + g;
   const uint32_t* bits = reinterpret_cast<const uint32_t*>(dt) + bg * L;
   uint64_t* tau_g = plan.tau + bg * L;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = static_cast<int>(blockDim.x >> 5);
+  const uint32_t lt = lanemask_lt();
   const int t_first = blockIdx.x * tpc;
   const int t_last = min(plan.n_row_tiles, t_first + tpc);
-  bool have = false;      // the previous tile's union and last-row tau carry over
-  int cur = 0;            // buffer holding the previous tile's union
-  int nU_prev = 0, q_prev = 0;
-  uint64_t tau_last = 0ull;
+  bool have = false;      // K(q') of the previous tile and this tile's tau0 carry over
+  int cur = 0;            // buffer whose head holds K
+  int q_prev = 0;
+  uint64_t tau0 = 0ull;
+  uint32_t pre_bits = 0u;   // dt bits of this tile's new key q' + 1 + tid (prefetched)
 
   for (int t = t_first; t < t_last; ++t) {
     const int r0 = t * kRowTile;
@@ -152,133 +529,260 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_prefill_kernel(const fl
       continue;
     }
 
-    uint64_t* U = Ubuf + (cur ^ 1) * ucap;
-    int nU;
-    if (have) {
-      // 1. threshold at the first row from the previous tile's last kept set
-      const uint64_t* Up = Ubuf + cur * ucap;
-      uint64_t tau0 = tau_last;
-      if (p != q_prev) {   // p == q_prev + 1: one new key competes
-        const uint64_t nk = composite_key(bits[p], static_cast<uint32_t>(p));
-        const uint64_t a2 = block_min_above(Up, nU_prev, tau_last, sm.bot_raw);   // second worst kept key
-        tau0 = nk < tau_last ? tau_last : (nk < a2 ? nk : a2);
-      }
-      // 2. the union: kept keys of the previous union, then the new keys (q_prev, q]
-      const int n_new = q - q_prev;
-      nU = ordered_compact(
-          nU_prev + n_new,
-          [&](int e) {
-            const uint64_t k = e < nU_prev ? Up[e]
-                                           : composite_key(bits[q_prev + 1 + (e - nU_prev)],
-                                                           static_cast<uint32_t>(q_prev + 1 + (e - nU_prev)));
-            return k >= tau0;
-          },
-          [&](int pos, int e) {
-            U[pos] = e < nU_prev ? Up[e]
-                                 : composite_key(bits[q_prev + 1 + (e - nU_prev)],
-                                                 static_cast<uint32_t>(q_prev + 1 + (e - nU_prev)));
-          },
-          sc);
-    } else {
-      // 1. threshold at the first row over its prefix
-      uint64_t tau0 = 0ull;
-      if (p + 1 > w) tau0 = select_kth_global(bits, p + 1, static_cast<uint32_t>(w), sc);
-      // 2. the union U of kept keys, in index order
-      nU = ordered_compact_row(
-          bits, q + 1, [&](uint32_t v, int j) { return composite_key(v, j) >= tau0; },
-          [&](int pos, int j, uint32_t v) { U[pos] = composite_key(v, j); }, sc);
-    }
-    __syncthreads();
-    const int n_old = p + 1 > w ? w : p + 1;
+    // the next tile of the run: its first row, last row and new keys (q, q_next],
+    // whose dt loads are issued now and used one tile later
+    const bool more = t + 1 < t_last;
+    const int p_next = min(r0 + kRowTile, len - 1);
+    const int q_next = more ? min(r0 + kRowTile + min(kRowTile, L - r0 - kRowTile) - 1, len - 1) : q;
+    uint32_t pre_next = 0u;
+    if (more && tid < q_next - q) pre_next = __ldg(bits + q + 1 + tid);
 
-    // 3. the kRowTile smallest keys of U, ascending; then tau for every row
-    const int nbot = min(nU, kRowTile);
-    uint64_t sigma = ~0ull;
-    if (nU > kRowTile) sigma = select_kth_smem(U, nU, static_cast<uint32_t>(nU - kRowTile + 1), sc);
-    if (tid == 0) sm.misc[0] = 0;
+    // K, the kept set at p (tau0 and above, at or before p), sorted, in buffer cur
+    int n_keep, j_new;   // keys of K at or above tau0; the new keys are (j_new, q]
+    uint32_t new_bits;
+    if (have) {
+      uint64_t* K = Ubuf + static_cast<size_t>(cur) * ucap;
+      n_keep = K[w - 1] >= tau0 ? w : w - 1;   // only the smallest key can fall below tau0
+      j_new = q_prev;
+      new_bits = pre_bits;
+    } else {
+      // K(p) = the keys at or before p at or above tau0 (the w-th largest), then sorted
+      tau0 = 0ull;
+      unsigned long long* ctr = reinterpret_cast<unsigned long long*>(&sm.vars[6]);
+      if (p + 1 > w && prefix_topw(bits, p + 1, w, Ubuf, 2 * ucap, sc, ctr, &tau0)) {
+        n_keep = w;
+      } else {
+        if (p + 1 > w) tau0 = select_kth_global(bits, p + 1, static_cast<uint32_t>(w), sc);
+        n_keep = row_collect_ge(bits, p + 1, tau0, Ubuf, ucap, ctr);
+      }
+      if (!block_bucket_sort_desc(Ubuf, Ubuf + ucap, n_keep, sm.hist, sm.red)) block_bitonic_desc(Ubuf, n_keep);
+      cur = 0;
+      j_new = p;
+      new_bits = (tid < q - p) ? __ldg(bits + p + 1 + tid) : 0u;
+    }
+    uint64_t* K = Ubuf + static_cast<size_t>(cur) * ucap;
+    uint64_t* U = Ubuf + static_cast<size_t>(cur ^ 1) * ucap;
+
+    // the new keys (j_new, q] at or above tau0, sorted: rank among them by count
+    const int n_new = q - j_new;
+    uint64_t nkey = 0ull;
+    if (tid < n_new) {
+      nkey = composite_key(new_bits, static_cast<uint32_t>(j_new + 1 + tid));
+      if (nkey < tau0) nkey = 0ull;
+    }
+    if (tid < kRowTile) {
+      sm.newk[tid] = nkey;
+      const uint32_t v = __ballot_sync(0xFFFFFFFFu, nkey != 0ull);
+      if (lane == 0) sm.cnt[0][warp] = __popc(v);
+    }
+    if (tid < kRowTile / 32) {
+      sm.newmask[tid] = 0u;
+      sm.oldmask[tid] = 0u;
+    }
+    if (tid == 0 && more) sm.nextk = composite_key(pre_next, static_cast<uint32_t>(p_next));
     __syncthreads();
-    for (int e = tid; e < nU; e += blockDim.x) {
-      if (U[e] <= sigma) {
-        const int pos = atomicAdd(&sm.misc[0], 1);
-        if (pos < kRowTile) sm.bot_raw[pos] = U[e];
+    int n_pass = 0;
+#pragma unroll
+    for (int k = 0; k < kRowTile / 32; ++k) n_pass += static_cast<int>(sm.cnt[0][k]);
+    if (nkey != 0ull) {
+      int rank = 0;
+#pragma unroll 16
+      for (int m = 0; m < kRowTile; ++m) rank += sm.newk[m] > nkey;
+      sm.news[rank] = nkey;
+      const int o = j_new + 1 + tid - r0;   // row offset of a key newer than the first row
+      if (o >= 1 && o < kRowTile) atomicOr(&sm.newmask[o >> 5], 1u << (o & 31));
+    }
+    __syncthreads();
+
+    // U = merge of K's first n_keep keys and the sorted new keys: each new key's
+    // insertion point in K, then each key of K shifts by the new keys above it
+    if (tid < n_pass) sm.ins[tid] = count_greater(K, n_keep, sm.news[tid]);
+    __syncthreads();
+    {
+      int insl[kRowTile / 32];   // lane l holds ins[l + 32 k] (n_keep + 1 past the end: never counted)
+#pragma unroll
+      for (int k = 0; k < kRowTile / 32; ++k) insl[k] = lane + 32 * k < n_pass ? sm.ins[lane + 32 * k] : n_keep + 1;
+      for (int e0 = warp * 32; e0 < n_keep; e0 += nw * 32) {
+        int c0 = 0;   // new keys inserted at or before e0
+#pragma unroll
+        for (int k = 0; k < kRowTile / 32; ++k) c0 += __popc(__ballot_sync(0xFFFFFFFFu, insl[k] <= e0));
+        const int e = e0 + lane;
+        int c = c0;
+        for (int m = c0; m < n_pass && sm.ins[m] <= e0 + 31; ++m) c += sm.ins[m] <= e;
+        if (e < n_keep) U[e + c] = K[e];
+      }
+    }
+    if (tid < n_pass) U[tid + sm.ins[tid]] = sm.news[tid];
+    const int nU = n_keep + n_pass;
+    const int n_old = p + 1 > w ? w : p + 1;
+    const int nbot = min(nU, kRowTile);
+    if (tid < kRowTile) sm.rowpos[tid] = -1;
+    __syncthreads();
+
+    // the tail (nbot smallest keys of U, ascending position s = nU - 1 - e):
+    // keys every row sees, and the row at which each newer key appears
+    if (tid < kRowTile) {
+      bool old = false;
+      if (tid < nbot) {
+        const int j = static_cast<int>(composite_index(U[nU - 1 - tid]));
+        old = j <= r0;
+        if (!old && j - r0 < kRowTile) sm.rowpos[j - r0] = static_cast<int16_t>(tid);
+      }
+      const uint32_t v = __ballot_sync(0xFFFFFFFFu, old);
+      if (lane == 0) sm.oldmask[warp] = v;
+    }
+    __syncthreads();
+    // tau of every row: the rank-th set bit of (old tail keys | tail keys new by this row)
+    uint32_t vis[kRowTile / 32] = {0u, 0u, 0u, 0u};
+    if (tid < kRowTile) {
+      const int rp = sm.rowpos[tid];
+      if (rp >= 0) vis[rp >> 5] = 1u << (rp & 31);
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+#pragma unroll
+        for (int k = 0; k < kRowTile / 32; ++k) {
+          const uint32_t x = __shfl_up_sync(0xFFFFFFFFu, vis[k], d);
+          if (lane >= d) vis[k] |= x;
+        }
+      }
+      if (lane == 31) {
+#pragma unroll
+        for (int k = 0; k < kRowTile / 32; ++k) sm.wor[warp][k] = vis[k];
       }
     }
     __syncthreads();
-    if (tid < nbot) {
-      const uint64_t key = sm.bot_raw[tid];
-      int rank = 0;
-      for (int f = 0; f < nbot; ++f) rank += sm.bot_raw[f] < key;
-      sm.bot[rank] = key;
-    }
-    __syncthreads();
-    if (tid < kRowTile) {
-      uint64_t tau = ~0ull;   // rows past the end of the sequence axis: unused
-      if (tid < nrows) {
-        const int ip = min(r0 + tid, len - 1);
-        if (ip + 1 <= w) {
-          tau = 0ull;
-        } else {
-          // keys of U visible to this row: the n_old old keys plus new keys j <= ip
-          int lo = n_old, hi = nU;
-          while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (static_cast<int>(composite_index(U[mid])) <= ip) lo = mid + 1; else hi = mid;
-          }
-          const int rank = lo - w + 1;   // ascending rank of the row's w-th best key
-          int c = 0;
-          tau = 0ull;
-          for (int e = 0; e < nbot; ++e) {
-            const uint64_t key = sm.bot[e];
-            if (static_cast<int>(composite_index(key)) <= ip && ++c == rank) {
-              tau = key;
-              break;
-            }
+    if (tid < nrows) {
+      for (int ww = 0; ww < warp; ++ww) {
+#pragma unroll
+        for (int k = 0; k < kRowTile / 32; ++k) vis[k] |= sm.wor[ww][k];
+      }
+      const int ip = min(r0 + tid, len - 1);
+      uint64_t tau = 0ull;
+      int pos = -1;
+      if (ip + 1 > w) {
+        int rank = n_old + popc_upto(sm.newmask, ip - r0) - w + 1;
+#pragma unroll
+        for (int k = 0; k < kRowTile / 32; ++k) {
+          const uint32_t v = vis[k] | sm.oldmask[k];
+          const int c = __popc(v);
+          if (pos < 0) {
+            if (rank <= c) pos = 32 * k + nth_set_bit(v, rank);
+            else rank -= c;
           }
         }
-        tau_g[r0 + tid] = tau;
+        if (pos < 0 || pos >= nbot) pos = nbot - 1;   // unreachable: every row's tau is a visible tail key
+        tau = U[nU - 1 - pos];
       }
+      tau_g[r0 + tid] = tau;
       sm.tau_s[tid] = tau;
+      sm.pos_s[tid] = pos;
     }
     __syncthreads();
 
-    // 4. row intervals and the two-class ordered list
-    const int per = (nU + blockDim.x - 1) / blockDim.x;
-    const int e0 = tid * per, e1 = min(nU, e0 + per);
-    uint32_t nf = 0, np = 0;
-    for (int e = e0; e < e1; ++e) {
-      const uint64_t key = U[e];
-      const int j = static_cast<int>(composite_index(key));
-      const int lo = j > r0 ? j - r0 : 0;
-      int a = 0, c = nrows;   // first row whose tau exceeds the key
-      while (a < c) {
-        const int mid = (a + c) >> 1;
-        if (sm.tau_s[mid] > key) c = mid; else a = mid + 1;
+    // each tail key is kept up to the first row whose tau lies above it; the
+    // tail decides the class sizes (a key above the tail is kept from its row
+    // to the end of the tile): n_full = keys seen by every row minus those of
+    // them evicted in the tile, the rest = newer keys kept by some row plus the
+    // evicted ones
+    if (tid < kRowTile) {
+      bool ev_old = false, dead_new = false;
+      if (tid < nbot) {
+        int a = 0, c = nrows;
+        while (a < c) {
+          const int mid = (a + c) >> 1;
+          if (sm.pos_s[mid] <= tid) a = mid + 1; else c = mid;
+        }
+        sm.hi_tail[tid] = static_cast<uint8_t>(a);
+        const int j = static_cast<int>(composite_index(U[nU - 1 - tid]));
+        const int lo = j > r0 ? j - r0 : 0;
+        ev_old = lo == 0 && a < nrows;
+        dead_new = lo > 0 && a <= lo;
       }
-      const int hi = a;
-      if (hi > lo) {
-        if (lo == 0 && hi == nrows) ++nf; else ++np;
+      const uint32_t v1 = __ballot_sync(0xFFFFFFFFu, ev_old), v2 = __ballot_sync(0xFFFFFFFFu, dead_new);
+      if (lane == 0) {
+        sm.cnt[0][warp] = __popc(v1);
+        sm.cnt[1][warp] = __popc(v2);
       }
     }
-    uint32_t total;
-    const uint32_t base = block_exclusive_scan(nf | (np << 16), sm.red, &total);
-    const int n_full = static_cast<int>(total & 0xFFFFu);
-    const int n_total = n_full + static_cast<int>(total >> 16);
-    uint32_t pf = base & 0xFFFFu, pp = n_full + (base >> 16);
-    for (int e = e0; e < e1; ++e) {
-      const uint64_t key = U[e];
-      const int j = static_cast<int>(composite_index(key));
-      const int lo = j > r0 ? j - r0 : 0;
-      int a = 0, c = nrows;
-      while (a < c) {
-        const int mid = (a + c) >> 1;
-        if (sm.tau_s[mid] > key) c = mid; else a = mid + 1;
+    if (tid == 0) {
+      sm.tot[2] = 0u;
+      sm.tot[3] = 0u;
+    }
+    // the next tile's tau0: the w-th largest of K(q) = U[0, w) and the key of its first row
+    uint64_t tau0n = 0ull;
+    if (more) {
+      const uint64_t tau_last = U[w - 1];
+      tau0n = tau_last;
+      if (p_next != q) {
+        const uint64_t a2 = w >= 2 ? U[w - 2] : ~0ull;
+        const uint64_t nk = sm.nextk;
+        tau0n = nk < tau_last ? tau_last : (nk < a2 ? nk : a2);
       }
-      const int hi = a;
-      if (hi > lo) {
-        const uint32_t pos = (lo == 0 && hi == nrows) ? pf++ : pp++;
-        idx_o[pos] = j;
-        bias_o[pos] = __uint_as_float(static_cast<uint32_t>(key >> 32));
-        span_o[pos] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+    }
+    __syncthreads();
+    int n_ev = 0, n_dead = 0;
+#pragma unroll
+    for (int k = 0; k < kRowTile / 32; ++k) {
+      n_ev += static_cast<int>(sm.cnt[0][k]);
+      n_dead += static_cast<int>(sm.cnt[1][k]);
+    }
+    const int n_lo0 = nU - static_cast<int>(__popc(sm.newmask[0]) + __popc(sm.newmask[1]) + __popc(sm.newmask[2]) +
+                                              __popc(sm.newmask[3]));   // keys at or before r0
+    const int n_full = n_lo0 - n_ev;
+    const int n_total = n_full + (nU - n_lo0) - n_dead + n_ev;
+
+    // the list: keys every row keeps, then the others.  Each warp takes a
+    // contiguous segment of U, counts its keys of both classes, reserves room
+    // for them with one atomic per class, then writes them.
+    int32_t* stage = reinterpret_cast<int32_t*>(K);   // K is dead once U is built
+    {
+      const int seg = ((nU + nw - 1) / nw + 31) / 32 * 32;
+      const int s0 = warp * seg, s1 = min(nU, s0 + seg);
+      auto classify = [&](int e, uint64_t& key, int& lo, int& hi, bool& f, bool& pp) {
+        key = U[e];
+        const int j = static_cast<int>(composite_index(key));
+        lo = j > r0 ? j - r0 : 0;
+        const int s_ = nU - 1 - e;
+        hi = s_ < nbot ? static_cast<int>(sm.hi_tail[s_]) : nrows;
+        f = lo == 0 && hi == nrows;
+        pp = !f && hi > lo;
+      };
+      uint32_t cf = 0, cp = 0;
+      for (int j0 = s0; j0 < s1; j0 += 32) {
+        const int e = j0 + lane;
+        uint64_t key = 0ull;
+        int lo = 0, hi = 0;
+        bool f = false, pp = false;
+        if (e < s1) classify(e, key, lo, hi, f, pp);
+        cf += __popc(__ballot_sync(0xFFFFFFFFu, f));
+        cp += __popc(__ballot_sync(0xFFFFFFFFu, pp));
+      }
+      uint32_t run_f = 0, run_p = 0;
+      if (lane == 0) {
+        if (cf) run_f = atomicAdd(&sm.tot[2], cf);
+        if (cp) run_p = atomicAdd(&sm.tot[3], cp);
+      }
+      run_f = __shfl_sync(0xFFFFFFFFu, run_f, 0);
+      run_p = __shfl_sync(0xFFFFFFFFu, run_p, 0) + static_cast<uint32_t>(n_full);
+      for (int j0 = s0; j0 < s1; j0 += 32) {
+        const int e = j0 + lane;
+        uint64_t key = 0ull;
+        int lo = 0, hi = 0;
+        bool f = false, pp = false;
+        if (e < s1) classify(e, key, lo, hi, f, pp);
+        const uint32_t vf = __ballot_sync(0xFFFFFFFFu, f), vp = __ballot_sync(0xFFFFFFFFu, pp);
+        if (f || pp) {
+          const uint32_t pos = f ? run_f + __popc(vf & lt) : run_p + __popc(vp & lt);
+          if (pos < static_cast<uint32_t>(ucap)) {
+            const int j = static_cast<int>(composite_index(key));
+            idx_o[pos] = j;
+            bias_o[pos] = __uint_as_float(static_cast<uint32_t>(key >> 32));
+            span_o[pos] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+            stage[pos] = j;
+          }
+        }
+        run_f += __popc(vf);
+        run_p += __popc(vp);
       }
     }
     const int padded = (n_total + kKeyTile - 1) / kKeyTile * kKeyTile;
@@ -288,27 +792,26 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_prefill_kernel(const fl
       span_o[j] = 0u;
     }
     if (tid == 0) plan.counts[tile] = make_int2(n_full, n_total);
+    __syncthreads();
     // key tiles whose listed keys are one ascending run j0, j0+1, ... can be
     // fetched with a single box copy instead of a row gather
-    __syncthreads();
     int32_t* kb = plan.kbase + tile * (plan.cap / kKeyTile);
-    const int lane = tid & 31;
-    for (int kt = tid >> 5; kt * kKeyTile < n_total; kt += blockDim.x >> 5) {
+    for (int kt = warp; kt * kKeyTile < n_total; kt += nw) {
       const int e0 = kt * kKeyTile;
-      const int j0 = idx_o[e0];
+      const int j0 = stage[e0];
       bool ok = true;
-      for (int e = e0 + lane; e < min(n_total, e0 + kKeyTile); e += 32) ok &= idx_o[e] == j0 + (e - e0);
+      for (int e = e0 + lane; e < min(n_total, e0 + kKeyTile); e += 32) ok &= stage[e] == j0 + (e - e0);
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (lane == 0) kb[kt] = ok ? j0 : -1;
     }
+    __syncthreads();   // the stage (in K's buffer) is read before the next tile writes there
 
-    // carried to the next tile: this union and the tau of its last visible row
-    tau_last = sm.tau_s[nrows - 1];
-    nU_prev = nU;
+    // carried to the next tile: K(q) = U[0, w) and its tau0
+    tau0 = tau0n;
     q_prev = q;
+    pre_bits = pre_next;
     cur ^= 1;
-    have = true;
-    __syncthreads();
+    have = more;
   }
 }
 
@@ -384,7 +887,15 @@ __global__ void decode_bitmask_kernel(DecodePlan plan, int Hkv, int Lk, uint32_t
   }
 }
 
-size_t select_smem_bytes(int ucap) { return sizeof(SelectSmem) + static_cast<size_t>(ucap) * sizeof(uint64_t); }
+size_t select_smem_bytes() { return sizeof(SelectSmem); }
+
+// prefill: the static part, then two key buffers of ucap keys (which also
+// hold the candidates of the prefix selection)
+size_t select_prefill_smem_bytes(int ucap) {
+  const size_t keys = static_cast<size_t>(ucap) * 2 > static_cast<size_t>(kCandCap) ? static_cast<size_t>(ucap) * 2
+                                                                                     : static_cast<size_t>(kCandCap);
+  return sizeof(PrefillSelSmem) + keys * sizeof(uint64_t);
+}
 
 }  // namespace
 
@@ -392,27 +903,30 @@ cudaError_t launch_select_prefill(const float* dt, const int32_t* lengths, const
                                   const PrefillPlan& plan, uint32_t* err, cudaStream_t s) {
   const int L = g.Lk;
   const int ucap = L > g.w ? g.w + kRowTile : 0;
-  const size_t smem = select_smem_bytes(2 * ucap);
+  const size_t smem = select_prefill_smem_bytes(ucap);
   cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(select_prefill_kernel), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  // row tiles per CTA: runs amortise the full selection, but the grid should
-  // still hold about four CTAs per SM (measured on the sparse and long
-  // workloads: 2 and 4 tiles per CTA); rows of 8 tiles or more use runs of at
-  // least 2
+  // row tiles per CTA: a run's first tile selects over its prefix and sorts
+  // its kept set, every later one only merges its new keys, so runs should be
+  // long; the grid should still fill one wave of resident CTAs with the tiles
+  // that need the top-k (rows below keep_window_size keep every visible key
+  // and cost little).  Measured on the sparse and long workloads: 3 and 8
+  // tiles per CTA (this rule gives 3 and 7).
   const int nsm = sm_count();
   if (nsm <= 0) return cudaErrorInvalidDevice;
-  const long long tiles = static_cast<long long>(plan.n_row_tiles) * g.Hkv * g.B;
-  long long tpc = (tiles + 4LL * nsm - 1) / (4LL * nsm);
-  if (plan.n_row_tiles >= 8 && tpc < 2) tpc = 2;
+  const long long free_tiles = L > g.w ? std::min<long long>(plan.n_row_tiles, g.w / kRowTile) : plan.n_row_tiles;
+  const long long topk_tiles = (static_cast<long long>(plan.n_row_tiles) - free_tiles) * g.Hkv * g.B;
+  const long long slots = static_cast<long long>(kSelPrefillMinBlocks) * nsm;
+  long long tpc = (topk_tiles + slots - 1) / slots;
   tpc = tpc < 1 ? 1 : (tpc > kSelTilesPerCtaMax ? kSelTilesPerCtaMax : tpc);
   dim3 grid(static_cast<unsigned>((plan.n_row_tiles + tpc - 1) / tpc), g.Hkv, g.B);
-  return launch_after(select_prefill_kernel, grid, dim3(kSelThreads), smem, s, dt, lengths, g.Hkv, L, g.w,
+  return launch_after(select_prefill_kernel, grid, dim3(kSelPrefillThreads), smem, s, dt, lengths, g.Hkv, L, g.w,
                       static_cast<int>(tpc), plan, err);
 }
 
 cudaError_t launch_select_decode(const float* dt, const int32_t* lengths, const Geometry& g,
                                  const DecodePlan& plan, uint32_t* err, cudaStream_t s) {
-  const size_t smem = select_smem_bytes(0);
+  const size_t smem = select_smem_bytes();
   cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(select_decode_kernel), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(g.Hkv, g.B);

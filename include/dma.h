@@ -113,8 +113,9 @@ DMA_API dma_status_t dma_dt_scores(const void* v, const float* W_dt, const float
  *     dt     [B, Hkv, L]        float32   (written by dma_forward_prefill when dt_in is NULL)
  *     tau    [B, Hkv, L]        uint64    row thresholds (as tau_out)
  *     idx    [tiles, cap]       int32     the keys any row of the tile keeps: first
- *                                         those every row keeps, then the others, each
- *                                         class in ascending key order
+ *                                         those every row keeps, then the others (in
+ *                                         index order when no row needs the top-k;
+ *                                         otherwise the order inside a class is free)
  *     bias   [tiles, cap]       float32   dt of the listed key
  *     span   [tiles, cap]       uint32    lo | hi << 16: the tile rows [lo, hi) keeping it
  *     counts [tiles]            int32 x2  (n_full, n_total): entries [0, n_full) are kept

@@ -30,8 +30,8 @@
 // every visible key and skip the selection; their lists are in index order.
 //
 // Decode (one CTA per (batch, kv head)): the single query at len_b - 1 keeps
-// the w best of its len_b keys; radix-select the w-th key, then compact the
-// kept keys in index order.
+// the w best of its len_b keys, selected and collected like a run's first
+// prefill tile and listed in any order.
 #include <algorithm>
 
 #include "select_common.cuh"
@@ -400,6 +400,7 @@ __device__ void row_collect2(const uint32_t* __restrict__ bits, int n, Cls cls, 
 // collects another way).  Every thread must call it.
 __device__ bool prefix_topw(const uint32_t* __restrict__ bits, int n, int w, uint64_t* out, int cap, SelScratch sc,
                             unsigned long long* counters, uint64_t* tau) {
+  if (w > cap) return false;
   uint32_t vor = 0u, vand = ~0u;
   row_for_each(bits, n, [&](uint32_t v, int, bool ok) {
     if (ok) {
@@ -815,7 +816,16 @@ __global__ void __launch_bounds__(kSelPrefillThreads, kSelPrefillMinBlocks) sele
   }
 }
 
-__global__ void __launch_bounds__(kSelThreads, 4) select_decode_kernel(const float* __restrict__ dt,
+// decode selector CTA: threads, and CTAs resident per SM (64 registers a thread)
+constexpr int kSelDecodeThreads = 256;
+constexpr int kSelDecodeMinBlocks = 4;
+
+// One CTA per (batch, kv head).  The w kept keys come from three passes over
+// the dt row (which bits vary, an 11-bit histogram, one collection of the keys
+// in and above the bin of the w-th largest), are finished in shared memory and
+// written from there; rows whose keys crowd one bin select and compact in two
+// more passes instead.
+__global__ void __launch_bounds__(kSelDecodeThreads, kSelDecodeMinBlocks) select_decode_kernel(const float* __restrict__ dt,
                                                                     const int32_t* __restrict__ lengths, int Hkv,
                                                                     int Lk, int w, DecodePlan plan, uint32_t* err) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -832,7 +842,15 @@ __global__ void __launch_bounds__(kSelThreads, 4) select_decode_kernel(const flo
   const int tid = threadIdx.x;
   int n;
   uint64_t tau = 0ull;
-  if (Lk > w && len > w) {
+  if (Lk > w && len > w && prefix_topw(bits, len, w, sm.cand, kCandCap, sc,
+                                       reinterpret_cast<unsigned long long*>(&sm.vars[6]), &tau)) {
+    n = w;
+    for (int e = tid; e < w; e += blockDim.x) {
+      const uint64_t key = sm.cand[e];
+      idx_o[e] = static_cast<int32_t>(composite_index(key));
+      bias_o[e] = __uint_as_float(static_cast<uint32_t>(key >> 32));
+    }
+  } else if (Lk > w && len > w) {
     tau = select_kth_global(bits, len, static_cast<uint32_t>(w), sc);
     n = ordered_compact_row(
         bits, len, [&](uint32_t v, int j) { return composite_key(v, j) >= tau; },
@@ -930,7 +948,7 @@ cudaError_t launch_select_decode(const float* dt, const int32_t* lengths, const 
   cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(select_decode_kernel), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(g.Hkv, g.B);
-  return launch_after(select_decode_kernel, grid, dim3(kSelThreads), smem, s, dt, lengths, g.Hkv, g.Lk, g.w, plan,
+  return launch_after(select_decode_kernel, grid, dim3(kSelDecodeThreads), smem, s, dt, lengths, g.Hkv, g.Lk, g.w, plan,
                       err);
 }
 

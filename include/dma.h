@@ -124,8 +124,8 @@ DMA_API dma_status_t dma_dt_scores(const void* v, const float* W_dt, const float
  *     kbase  [tiles, cap / 128] int32     j0 when 128-entry block k lists exactly
  *                                         j0, j0+1, ..., else -1
  *   Decode geometry (Lq == 1), cap = roundup(min(Lk, w), 128):
- *     dt [B, Hkv, Lk] float32, tau [B, Hkv] uint64, idx [B, Hkv, cap] int32 (kept
- *     keys ascending), bias [B, Hkv, cap] float32, count [B, Hkv] int32, then the
+ *     dt [B, Hkv, Lk] float32, tau [B, Hkv] uint64, idx [B, Hkv, cap] int32 (the
+ *     kept keys, in any order), bias [B, Hkv, cap] float32, count [B, Hkv] int32, then the
  *     split-K partials of dma_decode_step.
  */
 DMA_API dma_status_t dma_build_mask(const float* dt, const int32_t* lengths, int B, int Hkv, int Lq, int Lk,

@@ -252,6 +252,35 @@ __global__ void __launch_bounds__(kDtTcThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tiles = (ntok + kDtTile - 1) / kDtTile;
 
+  // the producer (thread 0) sets up the barriers and issues the first
+  // kDtStages copies at once, so the weight split below overlaps their latency
+  int pt = blockIdx.x, pkc = 0, pgs = 0;   // producer cursor: tile, chunk, copies issued
+  auto issue = [&]() {
+    const int s = pgs % kDtStages;
+    mbar_arrive_expect_tx(full + s, T::kStageBytes);
+    tma_load_2d(sA + s * T::kStageBytes, &tmap_v, full + s, pkc * kDtChunk, pt * kDtTile);
+    ++pgs;
+    if (++pkc == T::kChunks) {
+      pkc = 0;
+      pt += gridDim.x;
+    }
+  };
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDtStages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(acc_full + b, 1);
+      mbar_init(acc_empty + b, 4);   // one arrival per epilogue warp
+    }
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmap_v);
+    while (pgs < kDtStages && pt < n_tiles) issue();
+  }
+
   // B = [W_hi | W_mid | W_lo | 0], row n = term * HKV + g, K-major over the channels
   for (int i = threadIdx.x; i < T::C * HKV; i += blockDim.x) {
     const int c = i / HKV, g = i % HKV;
@@ -269,20 +298,6 @@ __global__ void __launch_bounds__(kDtTcThreads, 1)
     *reinterpret_cast<uint16_t*>(sB + b_offset<T::N>(n, c)) = 0;
   }
   fence_proxy_async_smem();
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kDtStages; ++s) {
-      mbar_init(full + s, 1);
-      mbar_init(empty + s, 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(acc_full + b, 1);
-      mbar_init(acc_empty + b, 4);   // one arrival per epilogue warp
-    }
-    mbar_init(fin, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) prefetch_tmap(&tmap_v);
   if (warp == 1) tmem_alloc(tmem_slot, T::kTmemCols);
   tc_fence_before();
   __syncthreads();
@@ -291,27 +306,22 @@ __global__ void __launch_bounds__(kDtTcThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      int gs = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-        for (int kc = 0; kc < T::kChunks; ++kc, ++gs) {
-          const int s = gs % kDtStages;
-          if (gs >= kDtStages &&
-              !mbar_wait(empty + s, ((gs / kDtStages) - 1) & 1, err, kDevErrTimeoutBase + 20)) {
-            ok = false;
-            *abort_flag = 1;
-            break;
-          }
-          if (aborted_flag(abort_flag)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(full + s, T::kStageBytes);
-          tma_load_2d(sA + s * T::kStageBytes, &tmap_v, full + s, kc * kDtChunk, t * kDtTile);
+      while (ok && pt < n_tiles) {
+        const int s = pgs % kDtStages;
+        if (!mbar_wait(empty + s, ((pgs / kDtStages) - 1) & 1, err, kDevErrTimeoutBase + 20)) {
+          ok = false;
+          *abort_flag = 1;
+          break;
         }
+        if (aborted_flag(abort_flag)) {
+          ok = false;
+          break;
+        }
+        issue();
       }
       // every copy issued must land before the CTA leaves
-      for (int j = gs - kDtStages < 0 ? 0 : gs - kDtStages; j < gs; ++j)
+      for (int j = pgs - kDtStages < 0 ? 0 : pgs - kDtStages; j < pgs; ++j)
         mbar_wait(full + j % kDtStages, (j / kDtStages) & 1, err, kDevErrTimeoutBase + 21);
     }
   } else if (warp == 1) {

@@ -217,6 +217,8 @@ struct RouteSmem {
   float wt[kMaxTopK];                   // routing weight * silu(h . down) per kept expert
   int ex[kMaxTopK];                     // kept experts, best first
   float sc[kMaxTopK];
+  int coff[kMaxTopK + 1];               // first candidate pair of each x key
+  float mout;                           // best pair score outside the candidate region
 };
 
 __device__ __forceinline__ float dot_bf16x8(uint4 a, uint4 b) {
@@ -230,21 +232,28 @@ __device__ __forceinline__ float dot_bf16x8(uint4 a, uint4 b) {
   return s;
 }
 
-// Keeps the k best of the domain's K keys: writes their scores and indices
-// (in no particular order) to (s_out, i_out).  Every thread must call it.
-__device__ __forceinline__ void domain_topk(const float* __restrict__ lg, int K, int k, RouteSmem& sm, SelScratch sc,
+// Keeps the k best of the domain's K <= blockDim keys, best first: thread j
+// ranks key j by counting the keys above it (composite keys are distinct) and
+// writes its score and index at that rank when the rank is below k.  Every
+// thread must call it.
+__device__ __forceinline__ void domain_topk(const float* __restrict__ lg, int K, int k, RouteSmem& sm,
                                             float* s_out, int* i_out) {
-  for (int j = threadIdx.x; j < K; j += blockDim.x)
-    sm.keys[j] = (static_cast<uint64_t>(ordered_bits(lg[j])) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(j));
+  uint64_t mine = 0ull;
+  if (static_cast<int>(threadIdx.x) < K) {
+    mine = (static_cast<uint64_t>(ordered_bits(lg[threadIdx.x])) << 32) | (0xFFFFFFFFu - threadIdx.x);
+    sm.keys[threadIdx.x] = mine;
+  }
   __syncthreads();
-  const uint64_t tau = select_kth_smem(sm.keys, K, static_cast<uint32_t>(k), sc);
-  ordered_compact(
-      K, [&](int j) { return sm.keys[j] >= tau; },
-      [&](int pos, int j) {
-        s_out[pos] = lg[j];
-        i_out[pos] = j;
-      },
-      sc);
+  if (static_cast<int>(threadIdx.x) < K) {
+    int rank = 0;
+#pragma unroll 8
+    for (int q = 0; q < K; ++q) rank += sm.keys[q] > mine;
+    if (rank < k) {
+      s_out[rank] = lg[threadIdx.x];
+      i_out[rank] = static_cast<int>(threadIdx.x);
+    }
+  }
+  __syncthreads();
 }
 
 __global__ void __launch_bounds__(kRouteThreads)
@@ -258,32 +267,87 @@ __global__ void __launch_bounds__(kRouteThreads)
   const int t = blockIdx.x;
   const float* lg = logits + static_cast<size_t>(t) * 2 * K;
 
-  // 1. the k best keys of each domain
-  domain_topk(lg, K, k, sm, sc, sm.sx, sm.ix);
-  domain_topk(lg + K, K, k, sm, sc, sm.sy, sm.iy);
-  // 2. the k best of the k * k pairs: float32 sum, expert a * K + b
-  const int n = k * k;
-  for (int p = threadIdx.x; p < n; p += blockDim.x) {
-    const int a = p / k, b = p - a * k;
-    const float s = sm.sx[a] + sm.sy[b];
-    const uint32_t e = static_cast<uint32_t>(sm.ix[a] * K + sm.iy[b]);
-    sm.keys[p] = (static_cast<uint64_t>(ordered_bits(s)) << 32) | (0xFFFFFFFFu - e);
+  // 1. the k best keys of each domain, best first
+  domain_topk(lg, K, k, sm, sm.sx, sm.ix);
+  domain_topk(lg + K, K, k, sm, sm.sy, sm.iy);
+  // 2. the k best pairs.  With both domains sorted, pair (a, b) is beaten by
+  // the (a+1)(b+1) pairs (a' <= a, b' <= b) at least as good, so the k best
+  // lie among the pairs with (a+1)(b+1) <= k (about k ln k of them): rank those
+  // by counting.  That is exact when the k-th of them scores strictly above
+  // every pair outside the region, whose best is sx[a] + sy[floor(k/(a+1))]
+  // for some a; otherwise (ties at the boundary) all k*k pairs are selected.
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int a = 0; a < k; ++a) {
+      sm.coff[a] = acc;
+      const int nb = k / (a + 1);
+      acc += nb < k ? nb : k;
+    }
+    sm.coff[k] = acc;
   }
   __syncthreads();
-  const uint64_t tau = select_kth_smem(sm.keys, n, static_cast<uint32_t>(k), sc);
-  ordered_compact(n, [&](int p) { return sm.keys[p] >= tau; }, [&](int pos, int p) { sm.fin[pos] = sm.keys[p]; },
-                  sc);
-  // 3. best first: rank of each kept key among the k (all distinct)
+  const int nc = sm.coff[k];
+  auto pair_key = [&](int a, int b) {
+    const float s = sm.sx[a] + sm.sy[b];
+    const uint32_t e = static_cast<uint32_t>(sm.ix[a] * K + sm.iy[b]);
+    return (static_cast<uint64_t>(ordered_bits(s)) << 32) | (0xFFFFFFFFu - e);
+  };
+  for (int c = threadIdx.x; c < nc; c += blockDim.x) {
+    int a = 0;
+    while (sm.coff[a + 1] <= c) ++a;
+    sm.keys[c] = pair_key(a, c - sm.coff[a]);
+  }
+  if (threadIdx.x < 32) {
+    // best score outside the region
+    float m = -INFINITY;
+    for (int a = threadIdx.x; a < k; a += 32) {
+      const int b = k / (a + 1);
+      if (b < k) m = fmaxf(m, sm.sx[a] + sm.sy[b]);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (threadIdx.x == 0) sm.mout = m;
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < nc; c += blockDim.x) {
+    const uint64_t mine = sm.keys[c];
+    int rank = 0;
+#pragma unroll 8
+    for (int q = 0; q < nc; ++q) rank += sm.keys[q] > mine;
+    if (rank < k) {
+      sm.fin[rank] = mine;
+      if (rank == k - 1) sm.vars[0] = mine;
+    }
+  }
+  __syncthreads();
+  const uint32_t ob_k = static_cast<uint32_t>(sm.vars[0] >> 32);
+  const bool exact = __uint_as_float((ob_k & 0x80000000u) ? (ob_k & 0x7FFFFFFFu) : ~ob_k) > sm.mout;
+  __syncthreads();
+  if (!exact) {
+    const int n = k * k;
+    for (int p = threadIdx.x; p < n; p += blockDim.x) sm.keys[p] = pair_key(p / k, p % k);
+    __syncthreads();
+    const uint64_t tau = select_kth_smem(sm.keys, n, static_cast<uint32_t>(k), sc);
+    ordered_compact(n, [&](int p) { return sm.keys[p] >= tau; }, [&](int pos, int p) { sm.fin[pos] = sm.keys[p]; },
+                    sc);
+    // best first: rank of each kept key among the k (all distinct)
+    uint64_t mine = 0ull;
+    if (threadIdx.x < k) mine = sm.fin[threadIdx.x];
+    int rank = 0;
+    if (threadIdx.x < k)
+      for (int q = 0; q < k; ++q) rank += sm.fin[q] > mine;
+    __syncthreads();
+    if (threadIdx.x < k) sm.fin[rank] = mine;
+    __syncthreads();
+  }
+  // 3. the kept experts and their scores, best first
   if (threadIdx.x < k) {
     const uint64_t mine = sm.fin[threadIdx.x];
-    int rank = 0;
-    for (int q = 0; q < k; ++q) rank += sm.fin[q] > mine;
     const int e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(mine & 0xFFFFFFFFull));
     // recover the float32 score from its ordered bits
     const uint32_t ob = static_cast<uint32_t>(mine >> 32);
-    const float s = __uint_as_float((ob & 0x80000000u) ? (ob & 0x7FFFFFFFu) : ~ob);
-    sm.ex[rank] = e;
-    sm.sc[rank] = s;
+    sm.ex[threadIdx.x] = e;
+    sm.sc[threadIdx.x] = __uint_as_float((ob & 0x80000000u) ? (ob & 0x7FFFFFFFu) : ~ob);
   }
   __syncthreads();
   if (experts_out && threadIdx.x < k) {

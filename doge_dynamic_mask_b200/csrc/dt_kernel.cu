@@ -281,17 +281,32 @@ __global__ void __launch_bounds__(kDtTcThreads, 1)
     while (pgs < kDtStages && pt < n_tiles) issue();
   }
 
-  // B = [W_hi | W_mid | W_lo | 0], row n = term * HKV + g, K-major over the channels
-  for (int i = threadIdx.x; i < T::C * HKV; i += blockDim.x) {
-    const int c = i / HKV, g = i % HKV;
-    const float w = W[i];
-    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
-    const float r1 = w - __bfloat162float(hi);
-    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
-    *reinterpret_cast<__nv_bfloat16*>(sB + b_offset<T::N>(g, c)) = hi;
-    *reinterpret_cast<__nv_bfloat16*>(sB + b_offset<T::N>(HKV + g, c)) = mid;
-    *reinterpret_cast<__nv_bfloat16*>(sB + b_offset<T::N>(2 * HKV + g, c)) = lo;
+  // B = [W_hi | W_mid | W_lo | 0], row n = term * HKV + g, K-major over the
+  // channels; each thread loads sixteen weights at a time, so their latencies
+  // overlap instead of adding up
+  constexpr int kWBatch = 16;
+  for (int i0 = 0; i0 < T::C * HKV; i0 += kWBatch * kDtTcThreads) {
+    float wv[kWBatch];
+#pragma unroll
+    for (int r = 0; r < kWBatch; ++r) {
+      const int i = i0 + r * kDtTcThreads + static_cast<int>(threadIdx.x);
+      wv[r] = i < T::C * HKV ? __ldg(W + i) : 0.0f;
+    }
+#pragma unroll
+    for (int r = 0; r < kWBatch; ++r) {
+      const int i = i0 + r * kDtTcThreads + static_cast<int>(threadIdx.x);
+      if (i < T::C * HKV) {
+        const int c = i / HKV, g = i % HKV;
+        const float w = wv[r];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+        const float r1 = w - __bfloat162float(hi);
+        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+        *reinterpret_cast<__nv_bfloat16*>(sB + b_offset<T::N>(g, c)) = hi;
+        *reinterpret_cast<__nv_bfloat16*>(sB + b_offset<T::N>(HKV + g, c)) = mid;
+        *reinterpret_cast<__nv_bfloat16*>(sB + b_offset<T::N>(2 * HKV + g, c)) = lo;
+      }
+    }
   }
   for (int i = threadIdx.x; i < (T::N - 3 * HKV) * T::C; i += blockDim.x) {
     const int n = 3 * HKV + i / T::C, c = i % T::C;

@@ -246,7 +246,7 @@ __device__ bool block_bucket_sort_desc(uint64_t* a, uint64_t* tmp, int n, uint32
 }
 
 // Appends, in any order, the composite keys of positions [0, n) of a dt row
-// that are >= tau to X (at most cap); returns their number.  Each warp
+// that are >= tau to X (at most cap are stored); returns their number.  Each warp
 // reserves room for sixteen keys per lane with one shared-memory atomic.
 // Every thread must call it.
 __device__ int row_collect_ge(const uint32_t* __restrict__ bits, int n, uint64_t tau, uint64_t* X, int cap,
@@ -307,7 +307,7 @@ __device__ int row_collect_ge(const uint32_t* __restrict__ bits, int n, uint64_t
   __syncthreads();
   const int r = static_cast<int>(*counter);
   __syncthreads();
-  return r < cap ? r : cap;
+  return r;   // may exceed cap (only cap keys were stored)
 }
 
 // Collects the composite keys of positions [0, n) of a dt row by class:
@@ -448,6 +448,39 @@ __device__ bool prefix_topw(const uint32_t* __restrict__ bits, int n, int w, uin
   return true;
 }
 
+constexpr int kSampleMax = 2048;
+
+// The keys of positions [0, n) of a dt row at or above a threshold t_lo that
+// lies a little below the w-th largest: t_lo is the r-th largest of kSampleMax
+// evenly spaced keys (r = 5/4 of w's share of the sample, plus 16), so about
+// 5/4 w keys pass.  One pass collects them into out (any order).  Returns
+// their number c; the caller uses them when w <= c <= cap (then the w-th
+// largest overall is the w-th largest among them), else falls back to an
+// exact selection.  Every thread must call it.
+__device__ int sampled_collect(const uint32_t* __restrict__ bits, int n, int w, uint64_t* out, int cap, SelScratch sc,
+                               unsigned long long* counter) {
+  const int S = n < kSampleMax ? n : kSampleMax;
+  if (S > cap) return -1;
+  for (int s0 = 0; s0 < S; s0 += 8 * blockDim.x) {   // eight independent loads in flight per thread
+    uint32_t v[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int s = s0 + r * blockDim.x + threadIdx.x;
+      v[r] = s < S ? __ldg(bits + static_cast<int>((static_cast<long long>(s) * n) / S)) : 0u;
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int s = s0 + r * blockDim.x + threadIdx.x;
+      if (s < S) out[s] = composite_key(v[r], static_cast<uint32_t>((static_cast<long long>(s) * n) / S));
+    }
+  }
+  __syncthreads();
+  long long r = (static_cast<long long>(w) * S * 5) / (static_cast<long long>(n) * 4) + 16;
+  if (r > S) r = S;
+  const uint64_t t_lo = select_kth_smem(out, S, static_cast<uint32_t>(r), sc);
+  return row_collect_ge(bits, n, t_lo, out, cap, counter);
+}
+
 // One CTA per (batch, kv head, run of tpc consecutive row tiles).
 //
 // The CTA keeps the union U of a tile (the keys any of its rows keeps) sorted
@@ -554,7 +587,7 @@ __global__ void __launch_bounds__(kSelPrefillThreads, kSelPrefillMinBlocks) sele
         n_keep = w;
       } else {
         if (p + 1 > w) tau0 = select_kth_global(bits, p + 1, static_cast<uint32_t>(w), sc);
-        n_keep = row_collect_ge(bits, p + 1, tau0, Ubuf, ucap, ctr);
+        n_keep = min(row_collect_ge(bits, p + 1, tau0, Ubuf, ucap, ctr), ucap);
       }
       if (!block_bucket_sort_desc(Ubuf, Ubuf + ucap, n_keep, sm.hist, sm.red)) block_bitonic_desc(Ubuf, n_keep);
       cur = 0;
@@ -820,11 +853,14 @@ __global__ void __launch_bounds__(kSelPrefillThreads, kSelPrefillMinBlocks) sele
 constexpr int kSelDecodeThreads = 256;
 constexpr int kSelDecodeMinBlocks = 4;
 
-// One CTA per (batch, kv head).  The w kept keys come from three passes over
-// the dt row (which bits vary, an 11-bit histogram, one collection of the keys
-// in and above the bin of the w-th largest), are finished in shared memory and
-// written from there; rows whose keys crowd one bin select and compact in two
-// more passes instead.
+// One CTA per (batch, kv head).  dt of a long cache row is read from memory,
+// not from L2, so passes over it count: a sampled threshold lets one pass
+// collect about 5/4 w keys that surely hold the w kept ones, which are then
+// selected in shared memory and written from there.  When the sample misjudges
+// (fewer than w or more than the buffer), three passes select exactly (which
+// bits vary, an 11-bit histogram, one collection of the keys in and above the
+// w-th largest's bin), and rows whose keys crowd one bin select and compact in
+// two more.
 __global__ void __launch_bounds__(kSelDecodeThreads, kSelDecodeMinBlocks) select_decode_kernel(const float* __restrict__ dt,
                                                                     const int32_t* __restrict__ lengths, int Hkv,
                                                                     int Lk, int w, DecodePlan plan, uint32_t* err) {
@@ -842,8 +878,31 @@ __global__ void __launch_bounds__(kSelDecodeThreads, kSelDecodeMinBlocks) select
   const int tid = threadIdx.x;
   int n;
   uint64_t tau = 0ull;
-  if (Lk > w && len > w && prefix_topw(bits, len, w, sm.cand, kCandCap, sc,
-                                       reinterpret_cast<unsigned long long*>(&sm.vars[6]), &tau)) {
+  int c = -1;
+  unsigned long long* ctr = reinterpret_cast<unsigned long long*>(&sm.vars[6]);
+  if (Lk > w && len > w) c = sampled_collect(bits, len, w, sm.cand, kCandCap, sc, ctr);
+  if (c >= w && c <= kCandCap) {
+    // the w-th largest among the collected keys, then the keys at or above it
+    tau = select_kth_smem(sm.cand, c, static_cast<uint32_t>(w), sc);
+    if (tid == 0) *ctr = 0ull;
+    __syncthreads();
+    const uint32_t lane = lane_id(), lt = lanemask_lt();
+    for (int e0 = 0; e0 < c; e0 += blockDim.x) {   // same trip count in every thread
+      const int e = e0 + tid;
+      const uint64_t key = e < c ? sm.cand[e] : 0ull;
+      const bool keep = e < c && key >= tau;
+      const uint32_t vote = __ballot_sync(0xFFFFFFFFu, keep);
+      uint32_t base = 0;
+      if (lane == 0 && vote) base = static_cast<uint32_t>(atomicAdd(ctr, static_cast<unsigned long long>(__popc(vote))));
+      base = __shfl_sync(0xFFFFFFFFu, base, 0);
+      if (keep) {
+        const uint32_t pos = base + __popc(vote & lt);
+        idx_o[pos] = static_cast<int32_t>(composite_index(key));
+        bias_o[pos] = __uint_as_float(static_cast<uint32_t>(key >> 32));
+      }
+    }
+    n = w;
+  } else if (Lk > w && len > w && prefix_topw(bits, len, w, sm.cand, kCandCap, sc, ctr, &tau)) {
     n = w;
     for (int e = tid; e < w; e += blockDim.x) {
       const uint64_t key = sm.cand[e];

@@ -14,9 +14,10 @@
 // Design.  Memory-bound: every projected row is read once and written once.
 // One CTA per token: the d/2 angles of its position are formed in double
 // precision (a position of 10^5 times a frequency near 1 would lose about
-// 2^-7 rad of its angle in float32, the size of a bf16 rounding) as turns,
-// reduced to their fractional part, and their cosines and sines taken in
-// float32 (sincospi) and kept in shared memory; then each group of d/8 lanes owns
+// 2^-7 rad of its angle in float32, the size of a bf16 rounding) as turns
+// (pos times theta^(-2i/d) / (2 pi), the factors formed once per call by the
+// launcher), reduced to their fractional part, and their cosines and sines
+// taken in float32 (sincospi) and kept in shared memory; then each group of d/8 lanes owns
 // one head row as sixteen-byte vectors (eight bf16 channels per lane): the
 // mean square is a group shuffle reduction, and channel i's rotation partner
 // i + d/2 sits in the lane d/16 positions away, one shuffle.  A lane's
@@ -50,10 +51,17 @@ struct RowPiece {
   int r;
 };
 
+// theta^(-2i/d) / (2 pi) for i < d/2: each angle in turns is pos times one of
+// these, formed once per call in double precision by the launcher
+struct RopeTurns {
+  double t[64];
+};
+
 template <int D>
 __global__ void __launch_bounds__(kPrologueThreads)
     prologue_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k, const uint4* __restrict__ v,
-                    const float* __restrict__ q_w, const float* __restrict__ k_w, float eps, double log_theta,
+                    const float* __restrict__ q_w, const float* __restrict__ k_w, float eps,
+                    const __grid_constant__ RopeTurns turns,
                     const int32_t* __restrict__ positions, int L, int Lmax, int Hq, int Hkv,
                     uint4* __restrict__ q_out, uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                     uint32_t* err) {
@@ -93,8 +101,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
     // the angle in turns, u = pos * theta^(-2i/d) / (2 pi), in double precision;
     // its fractional part r in [-1/2, 1/2] (exact in float32 to 2^-25) gives
     // cos and sin of 2 pi r = the angle modulo 2 pi, in float32
-    const double inv_freq = exp(-2.0 * static_cast<double>(threadIdx.x) / D * log_theta);
-    const double u = static_cast<double>(pos) * (inv_freq * 0.15915494309189535);   // 1 / (2 pi)
+    const double u = static_cast<double>(pos) * turns.t[threadIdx.x];
     const float r = static_cast<float>(u - rint(u));
     float sn, cs;
     sincospif(2.0f * r, &sn, &cs);
@@ -167,17 +174,20 @@ cudaError_t launch_prologue(const void* q, const void* k, const void* v, const f
                             int d, void* q_out, void* k_cache, void* v_cache, uint32_t* err, cudaStream_t s) {
   const long long tokens = static_cast<long long>(B) * L;
   if (tokens > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  if (d != 64 && d != 128) return cudaErrorInvalidValue;
+  RopeTurns turns{};
   const double log_theta = log(static_cast<double>(theta));
+  for (int i = 0; i < d / 2; ++i) turns.t[i] = exp(-2.0 * i / d * log_theta) * 0.15915494309189535;   // / (2 pi)
   const dim3 grid(static_cast<unsigned>(tokens)), block(kPrologueThreads);
   if (d == 64)
     prologue_kernel<64><<<grid, block, 0, s>>>(
         static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v), q_w, k_w, eps,
-        log_theta, positions, L, Lmax, Hq, Hkv, static_cast<uint4*>(q_out), static_cast<uint4*>(k_cache),
+        turns, positions, L, Lmax, Hq, Hkv, static_cast<uint4*>(q_out), static_cast<uint4*>(k_cache),
         static_cast<uint4*>(v_cache), err);
   else if (d == 128)
     prologue_kernel<128><<<grid, block, 0, s>>>(
         static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v), q_w, k_w, eps,
-        log_theta, positions, L, Lmax, Hq, Hkv, static_cast<uint4*>(q_out), static_cast<uint4*>(k_cache),
+        turns, positions, L, Lmax, Hq, Hkv, static_cast<uint4*>(q_out), static_cast<uint4*>(k_cache),
         static_cast<uint4*>(v_cache), err);
   else
     return cudaErrorInvalidValue;

@@ -398,7 +398,8 @@ __device__ void row_collect2(const uint32_t* __restrict__ bits, int n, Cls cls, 
 // B's keys at or above it join the front.  Returns false, with nothing
 // written, when B's keys would not fit beside the w (the caller selects and
 // collects another way).  Every thread must call it.
-__device__ bool prefix_topw(const uint32_t* __restrict__ bits, int n, int w, uint64_t* out, int cap, SelScratch sc,
+static __device__ __noinline__ bool prefix_topw(const uint32_t* __restrict__ bits, int n, int w, uint64_t* out, int cap,
+                                               SelScratch sc,
                             unsigned long long* counters, uint64_t* tau) {
   if (w > cap) return false;
   uint32_t vor = 0u, vand = ~0u;
@@ -448,12 +449,82 @@ __device__ bool prefix_topw(const uint32_t* __restrict__ bits, int n, int w, uin
   return true;
 }
 
-constexpr int kSampleMax = 2048;
+// Collects, in any order, the composite keys of positions [0, n) of a dt row
+// that are >= tau into out[0, cap): warp w appends to its own region of
+// cap / warps keys with a running offset (no atomics), and pads the rest of
+// the region with 0 (below every key).  The row is read as 16-byte pieces,
+// four per thread per step, with the next step's pieces prefetched into L2
+// before this step's are loaded.  Returns the number of keys, or -1 when some warp's
+// region overflowed.  Every thread must call it.
+static __device__ __noinline__ int row_collect_ge_regions(const uint32_t* __restrict__ bits, int n, uint64_t tau,
+                                                         uint64_t* out, int cap, uint32_t* red) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int lane = static_cast<int>(lane_id()), warp = tid >> 5, nw = nt >> 5;
+  const uint32_t lt = lanemask_lt();
+  const int rcap = cap / nw;
+  uint64_t* reg = out + warp * rcap;
+  int run = 0;   // keys this warp found (may pass rcap: then only rcap are stored)
+  auto put = [&](bool m, uint64_t key) {
+    const uint32_t vote = __ballot_sync(0xFFFFFFFFu, m);
+    if (m) {
+      const int pos = run + __popc(vote & lt);
+      if (pos < rcap) reg[pos] = key;
+    }
+    run += __popc(vote);
+  };
+  const bool vec = (reinterpret_cast<uintptr_t>(bits) & 15u) == 0;
+  const int nq = vec ? (n >> 2) : 0;
+  const uint4* qv = reinterpret_cast<const uint4*>(bits);
+  for (int r0 = 0; r0 < nq; r0 += 4 * nt) {   // same trip count in every thread
+    // the next step's pieces go to L2 now, so its loads do not wait on memory
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = r0 + 4 * nt + u * nt + tid;
+      if (i < nq) asm volatile("prefetch.global.L2 [%0];" ::"l"(qv + i));
+    }
+    uint4 cur[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = r0 + u * nt + tid;
+      cur[u] = i < nq ? __ldg(qv + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = r0 + u * nt + tid;
+      const bool ok = i < nq;
+      const uint32_t x[4] = {cur[u].x, cur[u].y, cur[u].z, cur[u].w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint64_t key = composite_key(x[c], static_cast<uint32_t>(4 * i + c));
+        put(ok && key >= tau, key);
+      }
+    }
+  }
+  for (int j0 = nq << 2; j0 < n; j0 += nt) {   // the rest of the row (or a row not 16-byte aligned)
+    const int j = j0 + tid;
+    const uint64_t key = j < n ? composite_key(__ldg(bits + j), static_cast<uint32_t>(j)) : 0ull;
+    put(j < n && key >= tau, key);
+  }
+  for (int e = run + lane; e < rcap; e += 32) reg[e] = 0ull;
+  if (lane == 0) red[warp] = static_cast<uint32_t>(run);
+  __syncthreads();
+  int total = 0;
+  bool over = false;
+  for (int k = 0; k < nw; ++k) {
+    total += static_cast<int>(red[k]);
+    over |= static_cast<int>(red[k]) > rcap;
+  }
+  __syncthreads();
+  return over ? -1 : total;
+}
+
+constexpr int kSampleMax = 4096;
 
 // The keys of positions [0, n) of a dt row at or above a threshold t_lo that
-// lies a little below the w-th largest: t_lo is the r-th largest of kSampleMax
-// evenly spaced keys (r = 5/4 of w's share of the sample, plus 16), so about
-// 5/4 w keys pass.  One pass collects them into out (any order).  Returns
+// lies a little below the w-th largest: t_lo is the r-th largest of a sample
+// of kSampleMax keys, 64 runs of 64 consecutive keys spread evenly over the
+// row (r = 3/2 of w's share of the sample, plus 16), so about 3/2 w keys pass
+// (for i.i.d. scores fewer than w is a 5.5 sigma event at the decode sizes).  One pass collects them into out (any order).  Returns
 // their number c; the caller uses them when w <= c <= cap (then the w-th
 // largest overall is the w-th largest among them), else falls back to an
 // exact selection.  Every thread must call it.
@@ -461,24 +532,27 @@ __device__ int sampled_collect(const uint32_t* __restrict__ bits, int n, int w, 
                                unsigned long long* counter) {
   const int S = n < kSampleMax ? n : kSampleMax;
   if (S > cap) return -1;
+  // the sample: 64 runs of 64 consecutive keys (two 128-byte lines each)
+  // spread evenly over the row, or the whole row when it is short
+  auto pos_of = [&](int s) { return S < kSampleMax ? s : (s >> 6) * (n / 64) + (s & 63); };
   for (int s0 = 0; s0 < S; s0 += 8 * blockDim.x) {   // eight independent loads in flight per thread
     uint32_t v[8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int s = s0 + r * blockDim.x + threadIdx.x;
-      v[r] = s < S ? __ldg(bits + static_cast<int>((static_cast<long long>(s) * n) / S)) : 0u;
+      v[r] = s < S ? __ldg(bits + pos_of(s)) : 0u;
     }
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int s = s0 + r * blockDim.x + threadIdx.x;
-      if (s < S) out[s] = composite_key(v[r], static_cast<uint32_t>((static_cast<long long>(s) * n) / S));
+      if (s < S) out[s] = composite_key(v[r], static_cast<uint32_t>(pos_of(s)));
     }
   }
   __syncthreads();
-  long long r = (static_cast<long long>(w) * S * 5) / (static_cast<long long>(n) * 4) + 16;
+  long long r = (static_cast<long long>(w) * S * 3) / (static_cast<long long>(n) * 2) + 16;
   if (r > S) r = S;
   const uint64_t t_lo = select_kth_smem(out, S, static_cast<uint32_t>(r), sc);
-  return row_collect_ge(bits, n, t_lo, out, cap, counter);
+  return row_collect_ge_regions(bits, n, t_lo, out, cap, sc.red);
 }
 
 // One CTA per (batch, kv head, run of tpc consecutive row tiles).
@@ -855,7 +929,7 @@ constexpr int kSelDecodeMinBlocks = 4;
 
 // One CTA per (batch, kv head).  dt of a long cache row is read from memory,
 // not from L2, so passes over it count: a sampled threshold lets one pass
-// collect about 5/4 w keys that surely hold the w kept ones, which are then
+// collect about 3/2 w keys that surely hold the w kept ones, which are then
 // selected in shared memory and written from there.  When the sample misjudges
 // (fewer than w or more than the buffer), three passes select exactly (which
 // bits vary, an 11-bit histogram, one collection of the keys in and above the
@@ -881,8 +955,10 @@ __global__ void __launch_bounds__(kSelDecodeThreads, kSelDecodeMinBlocks) select
   int c = -1;
   unsigned long long* ctr = reinterpret_cast<unsigned long long*>(&sm.vars[6]);
   if (Lk > w && len > w) c = sampled_collect(bits, len, w, sm.cand, kCandCap, sc, ctr);
-  if (c >= w && c <= kCandCap) {
-    // the w-th largest among the collected keys, then the keys at or above it
+  if (c >= w) {
+    // the w-th largest among the collected keys (the zero padding ranks last),
+    // then the keys at or above it
+    c = kCandCap;
     tau = select_kth_smem(sm.cand, c, static_cast<uint32_t>(w), sc);
     if (tid == 0) *ctr = 0ull;
     __syncthreads();

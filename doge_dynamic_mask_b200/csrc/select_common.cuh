@@ -21,7 +21,7 @@ namespace dma {
 
 constexpr int kSelThreads = 512;
 constexpr int kBins = 2048;      // 11-bit digits
-constexpr int kCandCap = 4096;   // shared-memory candidate buffer
+constexpr int kCandCap = 5632;   // shared-memory candidate buffer (704 keys per warp of a 256-thread CTA)
 
 struct SelScratch {
   uint32_t* hist;   // [kBins]

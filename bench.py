@@ -379,18 +379,21 @@ def time_prologue(dma, wl, steps, warmup, flush, dev, ranks_sync):
 
 def time_backward(dma, wl, steps, warmup, flush, dev, ranks_sync):
     """The backward of the prefill step (selection held fixed) on the
-    workload: dt, the kept-key lists, the attention backward and the dt chain."""
+    workload: dt, the kept-key lists, the attention backward and the dt chain.
+    The forward (run once, untimed) hands over out and each row's normaliser,
+    as a training step's forward does."""
     x = make_inputs(wl, device=dev)
     lengths = x["lengths"].cpu().numpy()
     out = torch.empty_like(x["q"])
-    dma.dma_forward_prefill(x["q"], x["k"], x["v"], x["W"], x["A"], x["lengths"], wl.w, out=out)
+    lse = torch.empty((wl.B, wl.Hq, wl.L), dtype=torch.float32, device=dev)
+    dma.dma_forward_prefill(x["q"], x["k"], x["v"], x["W"], x["A"], x["lengths"], wl.w, out=out, lse_out=lse)
     g = torch.Generator(device=dev).manual_seed(wl.seed + 100)
     dout = torch.randn(x["q"].shape, generator=g, device=dev).to(torch.bfloat16)
     ws = dma.new_workspace(dma.dma_backward_workspace_size(wl.B, wl.L, wl.Hq, wl.Hkv, wl.d, wl.w), dev)
 
     def step(i):
         dma.dma_backward_prefill(x["q"], x["k"], x["v"], x["W"], x["A"], x["lengths"], wl.w, out, dout,
-                                 workspace=ws)
+                                 workspace=ws, lse_in=lse)
 
     for i in range(warmup):
         step(i)
@@ -689,7 +692,7 @@ def run_ours(args):
             "ms_per_step": round(bms, 5), "frac_of_bf16_peak": round(bw["flops"] / (bms * 1e-3) / 1e12 /
                                                                       peaks["bf16_tflops"], 4),
             "stage_ms": [round(x_, 5) for x_ in bw["stage_ms"]],
-            "note": "backward of the headline workload (selection held fixed): dt, kept-key lists, attention "
+            "note": "backward of the headline workload (selection held fixed, row normalisers from the forward): dt, kept-key lists, attention "
                     "backward and dt chain; 10 d FLOPs per kept pair per query head"}
         result["gpu_launches"] += bw["launches"]
         del bw

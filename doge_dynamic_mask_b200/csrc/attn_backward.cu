@@ -16,7 +16,8 @@
 // tile, query head); thread r owns row r of the tile.  It walks the row tile's
 // kept-key list (the forward's plan, 128 keys per tile) twice:
 //   * pass 1 recomputes each row's softmax statistics (max and sum) from
-//     S = Q K^T + bias on the tensor core;
+//     S = Q K^T + bias on the tensor core, unless the forward pass handed
+//     over each row's log-sum-exp;
 //   * pass 2, per key tile: S = Q K^T and dP = dO V^T into TMEM; each thread
 //     forms its row of P and dS = P (dP - D) in float32 and stores them as bf16
 //     in shared memory (128-byte swizzle, [row][key]: the same bytes serve as
@@ -85,8 +86,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                     const __grid_constant__ CUtensorMap tmap_k3, const __grid_constant__ CUtensorMap tmap_v3,
                     PrefillPlan plan, int B, int L, int Hq, int Hkv, float scale, const uint16_t* __restrict__ out,
-                    const uint16_t* __restrict__ dout, uint16_t* __restrict__ dq, float* __restrict__ dk32,
-                    float* __restrict__ dv32, float* __restrict__ ddt32, uint32_t* err) {
+                    const uint16_t* __restrict__ dout, const float* __restrict__ lse_in, uint16_t* __restrict__ dq,
+                    float* __restrict__ dk32, float* __restrict__ dv32, float* __restrict__ ddt32, uint32_t* err) {
   using C = BwdCfg<D>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -258,16 +259,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   };
 
   // ---- pass 1: row statistics (log2 units): m = max, l = sum 2^(x - m) ----------
+  // (skipped when the forward pass handed over each row's log-sum-exp)
   float m = -INFINITY, l = 0.0f;
   int gs = 0;   // tiles loaded so far (both passes), for the ring phases
-  if (ok && n_kt > 0) load_tile(0, 0, false);
-  for (int j = 0; ok && j < n_kt; ++j, ++gs) {
+  const int n_kt1 = lse_in ? 0 : n_kt;
+  if (ok && n_kt1 > 0) load_tile(0, 0, false);
+  for (int j = 0; ok && j < n_kt1; ++j, ++gs) {
     const int s = gs % C::kStages;
     ok = mbar_wait(kv_full + s, phase_kv[s] & 1, err, kDevErrTimeoutBase + 42);
     phase_kv[s] ^= 1u;
     __syncthreads();   // the tile's metadata is visible to every thread
     // two stages: the other stage's tile (j - 1) is done, fetch tile j + 1 into it now
-    if (C::kStages == 2 && j + 1 < n_kt) load_tile(j + 1, (gs + 1) % C::kStages, false);
+    if (C::kStages == 2 && j + 1 < n_kt1) load_tile(j + 1, (gs + 1) % C::kStages, false);
     if (ok && tid == 0) {
       tc_fence_after();
       issue_xkt(q_lo, desc_lo(smem_u32(sK + s * C::kKVBytes), 16), 0);
@@ -304,9 +307,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     tc_fence_before();
     __syncthreads();   // S read by all before the next tile's MMA overwrites it
-    if (C::kStages == 1 && j + 1 < n_kt) load_tile(j + 1, (gs + 1) % C::kStages, false);
+    if (C::kStages == 1 && j + 1 < n_kt1) load_tile(j + 1, (gs + 1) % C::kStages, false);
   }
-  const float lse = (m == -INFINITY) ? 0.0f : m + log2f(l);
+  const float lse = lse_in ? (row_valid ? lse_in[(static_cast<size_t>(b) * Hq + h) * L + r0 + row] : 0.0f)
+                           : ((m == -INFINITY) ? 0.0f : m + log2f(l));
 
   // ---- pass 2: gradients ------------------------------------------------------
   if (ok && n_kt > 0) load_tile(0, gs % C::kStages, true);
@@ -533,8 +537,8 @@ __global__ void __launch_bounds__(kDtBwdThreads)
 
 template <int D>
 cudaError_t launch_bwd_d(const void* q, const void* k, const void* v, const void* out, const void* dout,
-                         const Geometry& g, float scale, const PrefillPlan& plan, void* dq, float* dk32, float* dv32,
-                         float* ddt32, uint32_t* err, cudaStream_t s) {
+                         const float* lse_in, const Geometry& g, float scale, const PrefillPlan& plan, void* dq,
+                         float* dk32, float* dv32, float* ddt32, uint32_t* err, cudaStream_t s) {
   using C = BwdCfg<D>;
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return cudaErrorNotSupported;
@@ -579,16 +583,16 @@ cudaError_t launch_bwd_d(const void* q, const void* k, const void* v, const void
   if (n_cta > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
   return launch_after(attn_bwd_kernel<D>, dim3(static_cast<unsigned>(n_cta)), dim3(kBwdThreads), C::kSmemBytes, s, tq,
                       tdo, tk, tv, tk3, tv3, plan, g.B, g.Lk, g.Hq, g.Hkv, scale, static_cast<const uint16_t*>(out),
-                      static_cast<const uint16_t*>(dout), static_cast<uint16_t*>(dq), dk32, dv32, ddt32, err);
+                      static_cast<const uint16_t*>(dout), lse_in, static_cast<uint16_t*>(dq), dk32, dv32, ddt32, err);
 }
 
 }  // namespace
 
 cudaError_t launch_attn_backward(const void* q, const void* k, const void* v, const void* out, const void* dout,
-                                 const Geometry& g, float scale, const PrefillPlan& plan, void* dq, float* dk32,
-                                 float* dv32, float* ddt32, uint32_t* err, cudaStream_t s) {
-  if (g.d == 64) return launch_bwd_d<64>(q, k, v, out, dout, g, scale, plan, dq, dk32, dv32, ddt32, err, s);
-  if (g.d == 128) return launch_bwd_d<128>(q, k, v, out, dout, g, scale, plan, dq, dk32, dv32, ddt32, err, s);
+                                 const float* lse_in, const Geometry& g, float scale, const PrefillPlan& plan,
+                                 void* dq, float* dk32, float* dv32, float* ddt32, uint32_t* err, cudaStream_t s) {
+  if (g.d == 64) return launch_bwd_d<64>(q, k, v, out, dout, lse_in, g, scale, plan, dq, dk32, dv32, ddt32, err, s);
+  if (g.d == 128) return launch_bwd_d<128>(q, k, v, out, dout, lse_in, g, scale, plan, dq, dk32, dv32, ddt32, err, s);
   return cudaErrorInvalidValue;
 }
 

@@ -248,7 +248,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_k3,
                         const __grid_constant__ CUtensorMap tmap_v3, PrefillPlan plan, int B, int L, int Hq,
-                        int Hkv, float scale_log2, float inv_scale, uint16_t* __restrict__ out, uint32_t* err) {
+                        int Hkv, float scale_log2, float inv_scale, uint16_t* __restrict__ out,
+                        float* __restrict__ lse_out, uint32_t* err) {
   using C = Cfg<D>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -870,8 +871,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = __all_sync(0xFFFFFFFFu, ok))) break;
       tc_fence_after();
       const float inv = 1.0f / l;
-      uint16_t* orow =
-          out + ((static_cast<size_t>(x.it.b) * L + r0 + row) * Hq + x.it.g * nrep + 2 * x.it.pair + h) * D;
+      const int head = x.it.g * nrep + 2 * x.it.pair + h;
+      uint16_t* orow = out + ((static_cast<size_t>(x.it.b) * L + r0 + row) * Hq + head) * D;
+      // the row's log-sum-exp in log2 units (m is the max the sum l was taken
+      // against), for a backward pass that reuses it; 0 for a row with no key
+      if (lse_out && row_valid)
+        lse_out[(static_cast<size_t>(x.it.b) * Hq + head) * L + r0 + row] = m == -INFINITY ? 0.0f : m + log2f(l);
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t o[32];
@@ -907,7 +912,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D>
 cudaError_t launch_d(const void* q, const void* k, const void* v, const Geometry& g, float scale,
-                     const PrefillPlan& plan, void* out, uint32_t* err, cudaStream_t s) {
+                     const PrefillPlan& plan, void* out, float* lse_out, uint32_t* err, cudaStream_t s) {
   using C = Cfg<D>;
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return cudaErrorNotSupported;
@@ -970,7 +975,7 @@ cudaError_t launch_d(const void* q, const void* k, const void* v, const Geometry
   const long long nblocks = n_items < nsm ? n_items : nsm;   // persistent: one CTA per SM
   return launch_after(attn_prefill_kernel<D>, dim3(static_cast<unsigned>(nblocks)), dim3(kThreads), C::kSmemBytes, s,
                       tq, tk, tv, tk3, tv3, plan, g.B, g.Lk, g.Hq, g.Hkv, scale * kLog2e, 1.0f / scale,
-                      static_cast<uint16_t*>(out), err);
+                      static_cast<uint16_t*>(out), lse_out, err);
 }
 
 }  // namespace
@@ -990,9 +995,9 @@ EncodeTiledFn get_encode_fn() {
 }
 
 cudaError_t launch_attn_prefill(const void* q, const void* k, const void* v, const Geometry& g, float scale,
-                                const PrefillPlan& plan, void* out, uint32_t* err, cudaStream_t s) {
-  if (g.d == 64) return launch_d<64>(q, k, v, g, scale, plan, out, err, s);
-  if (g.d == 128) return launch_d<128>(q, k, v, g, scale, plan, out, err, s);
+                                const PrefillPlan& plan, void* out, float* lse_out, uint32_t* err, cudaStream_t s) {
+  if (g.d == 64) return launch_d<64>(q, k, v, g, scale, plan, out, lse_out, err, s);
+  if (g.d == 128) return launch_d<128>(q, k, v, g, scale, plan, out, lse_out, err, s);
   return cudaErrorInvalidValue;
 }
 

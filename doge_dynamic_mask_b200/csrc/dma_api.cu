@@ -295,7 +295,16 @@ dma_status_t dma_forward_prefill(const void* q, const void* k, const void* v, co
                                  const int32_t* lengths, int B, int L, int Hq, int Hkv, int d, int keep_window_size,
                                  float scale, const float* dt_in, void* out, void* workspace, size_t ws_bytes,
                                  dma_stream_t stream) {
+  return dma_forward_prefill_lse(q, k, v, W_dt, A, lengths, B, L, Hq, Hkv, d, keep_window_size, scale, dt_in, out,
+                                 nullptr, workspace, ws_bytes, stream);
+}
+
+dma_status_t dma_forward_prefill_lse(const void* q, const void* k, const void* v, const float* W_dt, const float* A,
+                                     const int32_t* lengths, int B, int L, int Hq, int Hkv, int d,
+                                     int keep_window_size, float scale, const float* dt_in, void* out, float* lse_out,
+                                     void* workspace, size_t ws_bytes, dma_stream_t stream) {
   if (!q || !k || !v || !out || !workspace) return DMA_ERR_INVALID_ARG;
+  if (lse_out && !aligned16(lse_out)) return DMA_ERR_INVALID_ARG;
   if (!dt_in && (!W_dt || !A)) return DMA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace) ||
       (W_dt && !aligned16(W_dt)) || (A && !aligned16(A)) || (dt_in && !aligned16(dt_in)) ||
@@ -326,7 +335,7 @@ dma_status_t dma_forward_prefill(const void* q, const void* k, const void* v, co
   // each tile's key list (causal and padding bounds) itself
   if (!plan.no_topk && (e = launch_select_prefill(dt, lengths, g, plan, err, s)) != cudaSuccess) return cuda_fail(e);
   if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e);
-  if ((e = launch_attn_prefill(q, k, v, g, scale, plan, out, err, s)) != cudaSuccess) return cuda_fail(e);
+  if ((e = launch_attn_prefill(q, k, v, g, scale, plan, out, lse_out, err, s)) != cudaSuccess) return cuda_fail(e);
   if ((e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e);
   return DMA_OK;
 }
@@ -476,15 +485,15 @@ size_t dma_backward_workspace_size(int B, int L, int Hq, int Hkv, int d, int kee
 
 dma_status_t dma_backward_prefill(const void* q, const void* k, const void* v, const float* W_dt, const float* A,
                                   const int32_t* lengths, int B, int L, int Hq, int Hkv, int d, int keep_window_size,
-                                  float scale, const float* dt_in, const void* out, const void* dout, void* dq,
-                                  void* dk, void* dv, float* d_dt, float* dW_dt, float* dA, void* workspace,
-                                  size_t ws_bytes, dma_stream_t stream) {
+                                  float scale, const float* dt_in, const void* out, const void* dout,
+                                  const float* lse_in, void* dq, void* dk, void* dv, float* d_dt, float* dW_dt,
+                                  float* dA, void* workspace, size_t ws_bytes, dma_stream_t stream) {
   if (!q || !k || !v || !W_dt || !A || !out || !dout || !dq || !dk || !dv || !dW_dt || !dA || !workspace)
     return DMA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(W_dt) || !aligned16(A) || !aligned16(out) ||
       !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dW_dt) ||
       !aligned16(dA) || !aligned16(workspace) || (dt_in && !aligned16(dt_in)) || (d_dt && !aligned16(d_dt)) ||
-      (lengths && !aligned16(lengths)))
+      (lengths && !aligned16(lengths)) || (lse_in && !aligned16(lse_in)))
     return DMA_ERR_INVALID_ARG;
   if (!(scale >= 1.0e-20f && scale <= 1.0e20f)) return DMA_ERR_INVALID_ARG;
   dma_status_t st = check_shape(B, L, Hq, Hkv, d, keep_window_size);
@@ -517,7 +526,8 @@ dma_status_t dma_backward_prefill(const void* q, const void* k, const void* v, c
   // keep_window_size >= L (the lists then hold every visible key)
   if ((e = launch_select_prefill(dt, lengths, g, plan, err, s)) != cudaSuccess) return cuda_fail(e);
   if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e);
-  if ((e = launch_attn_backward(q, k, v, out, dout, g, scale, plan, dq, dk32, dv32, ddt32, err, s)) != cudaSuccess)
+  if ((e = launch_attn_backward(q, k, v, out, dout, lse_in, g, scale, plan, dq, dk32, dv32, ddt32, err, s)) !=
+      cudaSuccess)
     return cuda_fail(e);
   if ((e = launch_dt_backward(v, W_dt, A, ddt32, dk32, dv32, B, L, Hkv, d, dx, dW_dt, dA, dk, dv, s)) != cudaSuccess)
     return cuda_fail(e);

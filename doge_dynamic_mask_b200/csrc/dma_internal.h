@@ -138,8 +138,9 @@ cudaError_t launch_select_decode(const float* dt, const int32_t* lengths, const 
                                  const DecodePlan& plan, uint32_t* err, cudaStream_t s);
 cudaError_t launch_prefill_bitmask(const PrefillPlan& plan, const Geometry& g, uint32_t* bitmask, cudaStream_t s);
 cudaError_t launch_decode_bitmask(const DecodePlan& plan, const Geometry& g, uint32_t* bitmask, cudaStream_t s);
+// lse_out (may be null): float32 [B, Hq, L], each row's log-sum-exp in log2 units
 cudaError_t launch_attn_prefill(const void* q, const void* k, const void* v, const Geometry& g, float scale,
-                                const PrefillPlan& plan, void* out, uint32_t* err, cudaStream_t s);
+                                const PrefillPlan& plan, void* out, float* lse_out, uint32_t* err, cudaStream_t s);
 cudaError_t launch_attn_decode(const void* q, const void* k, const void* v, const Geometry& g, float scale,
                                const DecodePlan& plan, void* out, cudaStream_t s);
 // incremental decode: take in the tokens cached since the last step / finish a freshly selected state
@@ -158,9 +159,11 @@ cudaError_t launch_cdmoe_route_experts(const void* h, const float* logits, const
                                        int32_t* experts_out, float* scores_out, cudaStream_t s);
 // backward: attention with the selection held fixed (float32 dK / dV / d_dt
 // accumulators, zeroed by the caller), then the dt chain (dk / dv to bf16, dW, dA)
+// lse_in (may be null): the forward's row log-sum-exp [B, Hq, L] (log2 units);
+// when given, the backward skips recomputing the row statistics
 cudaError_t launch_attn_backward(const void* q, const void* k, const void* v, const void* out, const void* dout,
-                                 const Geometry& g, float scale, const PrefillPlan& plan, void* dq, float* dk32,
-                                 float* dv32, float* ddt32, uint32_t* err, cudaStream_t s);
+                                 const float* lse_in, const Geometry& g, float scale, const PrefillPlan& plan,
+                                 void* dq, float* dk32, float* dv32, float* ddt32, uint32_t* err, cudaStream_t s);
 cudaError_t launch_dt_backward(const void* v, const float* W, const float* A, const float* ddt32, const float* dk32,
                                const float* dv32, int B, int L, int Hkv, int d, float* dx, float* dW, float* dA,
                                void* dk, void* dv, cudaStream_t s);

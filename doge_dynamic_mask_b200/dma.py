@@ -34,6 +34,8 @@ _lib.dma_build_mask.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _sz
 _lib.dma_forward_prefill.restype = _i
 _lib.dma_forward_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _sz,
                                      _vp]
+_lib.dma_forward_prefill_lse.restype = _i
+_lib.dma_forward_prefill_lse.argtypes = [_vp] * 6 + [_i] * 6 + [_f] + [_vp] * 4 + [_sz, _vp]
 _lib.dma_decode_step.restype = _i
 _lib.dma_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _sz, _vp]
 _lib.dma_decode_state_size.restype = _sz
@@ -51,7 +53,7 @@ _lib.dma_cdmoe_forward.argtypes = [_vp] * 4 + [_i] * 4 + [_vp] * 5 + [_sz, _vp]
 _lib.dma_backward_workspace_size.restype = _sz
 _lib.dma_backward_workspace_size.argtypes = [_i] * 6
 _lib.dma_backward_prefill.restype = _i
-_lib.dma_backward_prefill.argtypes = [_vp] * 6 + [_i] * 6 + [_f] + [_vp] * 10 + [_sz, _vp]
+_lib.dma_backward_prefill.argtypes = [_vp] * 6 + [_i] * 6 + [_f] + [_vp] * 11 + [_sz, _vp]
 _lib.dma_selftest_wait.restype = _i
 _lib.dma_selftest_wait.argtypes = [_vp, _vp]
 _lib.dma_check.restype = _i
@@ -124,7 +126,9 @@ def dma_build_mask(dt, lengths, Lq, keep_window_size, workspace=None, tau_out=No
 
 
 def dma_forward_prefill(q, k, v, W_dt, A, lengths, keep_window_size, scale=None, dt_in=None, out=None,
-                        workspace=None, stream=None):
+                        workspace=None, stream=None, lse_out=None):
+    """With lse_out ([B, Hq, L] float32) the rows' normalisers are written too
+    (dma_forward_prefill_lse), for dma_backward_prefill(lse_in=...)."""
     B, L, Hq, d = q.shape
     Hkv = k.shape[2]
     if scale is None:
@@ -133,10 +137,16 @@ def dma_forward_prefill(q, k, v, W_dt, A, lengths, keep_window_size, scale=None,
         out = torch.empty_like(q)
     if workspace is None:
         workspace = new_workspace(dma_workspace_size(B, L, L, Hq, Hkv, d, keep_window_size), q.device)
-    _ok(_lib.dma_forward_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(W_dt), _ptr(A), _ptr(lengths), B, L, Hq, Hkv, d,
-                                 keep_window_size, float(scale), _ptr(dt_in), _ptr(out), _ptr(workspace),
-                                 workspace.numel(), _stream(stream)),
-        "dma_forward_prefill")
+    if lse_out is None:
+        _ok(_lib.dma_forward_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(W_dt), _ptr(A), _ptr(lengths), B, L, Hq, Hkv,
+                                     d, keep_window_size, float(scale), _ptr(dt_in), _ptr(out), _ptr(workspace),
+                                     workspace.numel(), _stream(stream)),
+            "dma_forward_prefill")
+    else:
+        _ok(_lib.dma_forward_prefill_lse(_ptr(q), _ptr(k), _ptr(v), _ptr(W_dt), _ptr(A), _ptr(lengths), B, L, Hq,
+                                         Hkv, d, keep_window_size, float(scale), _ptr(dt_in), _ptr(out),
+                                         _ptr(lse_out), _ptr(workspace), workspace.numel(), _stream(stream)),
+            "dma_forward_prefill_lse")
     return out
 
 
@@ -181,10 +191,11 @@ def dma_backward_workspace_size(B, L, Hq, Hkv, d, keep_window_size) -> int:
 
 
 def dma_backward_prefill(q, k, v, W_dt, A, lengths, keep_window_size, out, dout, scale=None, dt_in=None,
-                         workspace=None, want_d_dt=False, stream=None):
+                         workspace=None, want_d_dt=False, stream=None, lse_in=None):
     """Gradients of sum(out * dout) with the selection held fixed: returns
     (dq, dk, dv) bf16, dW_dt and dA float32, and d_dt [B, Hkv, L] float32 when
-    want_d_dt."""
+    want_d_dt.  lse_in: the forward's row normalisers (dma_forward_prefill with
+    lse_out), else they are recomputed."""
     B, L, Hq, d = q.shape
     Hkv = k.shape[2]
     if scale is None:
@@ -196,7 +207,8 @@ def dma_backward_prefill(q, k, v, W_dt, A, lengths, keep_window_size, out, dout,
     if workspace is None:
         workspace = new_workspace(dma_backward_workspace_size(B, L, Hq, Hkv, d, keep_window_size), q.device)
     _ok(_lib.dma_backward_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(W_dt), _ptr(A), _ptr(lengths), B, L, Hq, Hkv, d,
-                                  keep_window_size, float(scale), _ptr(dt_in), _ptr(out), _ptr(dout), _ptr(dq),
+                                  keep_window_size, float(scale), _ptr(dt_in), _ptr(out), _ptr(dout),
+                                  _ptr(lse_in), _ptr(dq),
                                   _ptr(dk), _ptr(dv), _ptr(d_dt), _ptr(dW), _ptr(dA), _ptr(workspace),
                                   workspace.numel(), _stream(stream)),
         "dma_backward_prefill")

@@ -148,6 +148,18 @@ DMA_API dma_status_t dma_forward_prefill(const void* q, const void* k, const voi
                                  dma_stream_t stream);
 
 /*
+ * As dma_forward_prefill, and also writes each query row's softmax
+ * normaliser for a later dma_backward_prefill:
+ *   lse_out  [B, Hq, L] float32 (16-byte aligned; written): log2 of the sum over
+ *            the row's kept keys of 2^((q.k * scale + dt) * log2(e)), i.e. the
+ *            natural log-sum-exp times log2(e); 0 for a row that keeps no key.
+ */
+DMA_API dma_status_t dma_forward_prefill_lse(const void* q, const void* k, const void* v, const float* W_dt,
+                                             const float* A, const int32_t* lengths, int B, int L, int Hq, int Hkv,
+                                             int d, int keep_window_size, float scale, const float* dt_in, void* out,
+                                             float* lse_out, void* workspace, size_t ws_bytes, dma_stream_t stream);
+
+/*
  * S4, [DMA step 3 closing paragraph, step 4]: one decode step.  dt is computed
  * over the whole cached value states, the query at position len_b - 1 keeps
  * its keep_window_size best cached keys, and attends to them as above.
@@ -203,6 +215,9 @@ DMA_API dma_status_t dma_prologue(const void* q, const void* k, const void* v, c
  * Arguments as dma_forward_prefill, plus:
  *   out      [B, L, Hq, d] bf16: the forward's output for the same inputs
  *   dout     [B, L, Hq, d] bf16: the gradient of the loss with respect to out
+ *   lse_in   [B, Hq, L] float32 or NULL: the forward's row normalisers
+ *            (dma_forward_prefill_lse); when NULL they are recomputed (one more
+ *            pass over every row tile's kept keys).
  *   dq       [B, L, Hq, d] bf16 (written);  dk, dv [B, L, Hkv, d] bf16 (written)
  *   d_dt     [B, Hkv, L] float32 (written) or NULL
  *   dW_dt    [Hkv*d, Hkv] float32 (written);  dA [Hkv] float32 (written)
@@ -216,9 +231,9 @@ DMA_API size_t dma_backward_workspace_size(int B, int L, int Hq, int Hkv, int d,
 DMA_API dma_status_t dma_backward_prefill(const void* q, const void* k, const void* v, const float* W_dt,
                                           const float* A, const int32_t* lengths, int B, int L, int Hq, int Hkv,
                                           int d, int keep_window_size, float scale, const float* dt_in,
-                                          const void* out, const void* dout, void* dq, void* dk, void* dv,
-                                          float* d_dt, float* dW_dt, float* dA, void* workspace, size_t ws_bytes,
-                                          dma_stream_t stream);
+                                          const void* out, const void* dout, const float* lse_in, void* dq,
+                                          void* dk, void* dv, float* d_dt, float* dW_dt, float* dA, void* workspace,
+                                          size_t ws_bytes, dma_stream_t stream);
 
 /*
  * CDMoE routing ([CDMoE], section "跨域 MoE（CDMoE）" of the same page): the

@@ -49,27 +49,31 @@ struct BwdCfg {
   static constexpr int kQBytes = kRowTile * D * 2;       // Q or dO tile
   static constexpr int kSlabBytes = kRowTile * 128;      // 128 rows x 64 bf16
   static constexpr int kKVBytes = kKeyTile * D * 2;
-  static constexpr int kPBytes = kRowTile * kKeyTile * 2; // P or dS: two 64-key chunks
-  static constexpr int kStages = D == 64 ? 2 : 1;
-  // Q, then the ones slab right after it (the B operand [Q | 1] spans both at one slab stride)
+  static constexpr int kPBytes = kRowTile * kKeyTile * 2; // P, then dS: two 64-key chunks
+  static constexpr int kStages = 1;
+  static constexpr int kOnesBytes = 16 * kRowTile * 2;    // the d_dt operand: 16 x 128 rows, K-major
   static constexpr int kOffQ = 0;
-  static constexpr int kOffOnes = kOffQ + kQBytes;
-  static constexpr int kOffDO = kOffOnes + kSlabBytes;
+  static constexpr int kOffDO = kOffQ + kQBytes;
   static constexpr int kOffK = kOffDO + kQBytes;
   static constexpr int kOffV = kOffK + kStages * kKVBytes;
   static constexpr int kOffP = kOffV + kStages * kKVBytes;
-  static constexpr int kOffDS = kOffP + kPBytes;
-  static constexpr int kOffMeta = kOffDS + kPBytes;       // per stage: bias[128] f32, span[128] u32, key[128] i32
+  static constexpr int kOffOnes = kOffP + kPBytes;
+  static constexpr int kOffMeta = kOffOnes + kOnesBytes;  // per stage: bias[128] f32, span[128] u32, key[128] i32
   static constexpr int kMetaBytes = 3 * kKeyTile * 4;
   static constexpr int kOffBar = kOffMeta + kStages * kMetaBytes;
   static constexpr int kSmemBytes = kOffBar + 128 + 1024;
-  // TMEM: S / dV_t at 0, dP / dK_t at 128 (dK_t is D + 64 wide: Q's columns
-  // and the whole ones slab, so the MN-major B operand is made of full
-  // 64-column swizzle atoms), dQ after it
-  static constexpr uint32_t kColDK = 128;
-  static constexpr uint32_t kColDQ = 128 + (D + 64 > 128 ? D + 64 : 128);
-  static_assert(kColDQ + D <= 512, "TMEM budget");
+  // TMEM: S, then dP, at [0, 128), then dK_t at [0, D) once dP is read;
+  // dV_t = P^T dO at [128, 128 + D); dQ after it; d_dt (16 columns, of which
+  // the first is used) in the free part of [0, 128) at d = 64, else after dQ
+  static constexpr uint32_t kColDK = 0;
+  static constexpr uint32_t kColDV = 128;
+  static constexpr uint32_t kColDQ = 128 + D;
+  static constexpr uint32_t kColDDT = D == 64 ? 64 : 128 + 2 * D;
+  static constexpr uint32_t kTmemCols = D == 64 ? 256 : 512;
+  static constexpr int kMinBlocks = D == 64 ? 2 : 1;     // d = 64: two CTAs share an SM (TMEM 2 x 256)
+  static_assert(kColDQ + D <= kTmemCols && kColDDT + 16 <= kTmemCols, "TMEM budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(D != 64 || 2 * (kSmemBytes + 1024) <= 233472, "two CTAs per SM at d = 64");
 };
 
 __device__ __forceinline__ float ld_bf16(const uint16_t* p) { return __uint_as_float(static_cast<uint32_t>(*p) << 16); }
@@ -81,7 +85,7 @@ __device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c
 }
 
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, BwdCfg<D>::kMinBlocks)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_do,
                     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                     const __grid_constant__ CUtensorMap tmap_k3, const __grid_constant__ CUtensorMap tmap_v3,
@@ -121,8 +125,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   unsigned char* sDO = smem + C::kOffDO;
   unsigned char* sK = smem + C::kOffK;
   unsigned char* sV = smem + C::kOffV;
-  unsigned char* sP = smem + C::kOffP;
-  unsigned char* sDS = smem + C::kOffDS;
+  unsigned char* sP = smem + C::kOffP;     // P, then dS, of the current key tile
   unsigned char* sMeta = smem + C::kOffMeta;
 
   if (tid == 0) {
@@ -133,17 +136,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     prefetch_tmap(&tmap_q);
     prefetch_tmap(&tmap_do);
   }
-  // the ones slab: column 0 of every row is 1, the rest 0 (128-byte swizzle)
+  // the d_dt operand, K-major over the tile's 128 rows: row n = 0 all ones,
+  // rows 1..15 zero (the 128-byte swizzle only permutes the 16-byte units of
+  // a row, and every unit of row 0 is alike), so column 0 of dS^T x it is the
+  // column sum of dS
   {
-    unsigned char* rowp = sOnes + row * 128;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const uint4 val = (u == (row & 7)) ? make_uint4(0x3F80u, 0u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
-      *reinterpret_cast<uint4*>(rowp + u * 16) = val;
-    }
+    const int kc = tid >> 6, n = (tid >> 2) & 15, u0 = (tid & 3) * 2;   // 128 threads x 32 bytes
+    const uint4 val = n == 0 ? make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u) : make_uint4(0u, 0u, 0u, 0u);
+    unsigned char* rowp = sOnes + kc * 2048 + n * 128;
+    *reinterpret_cast<uint4*>(rowp + u0 * 16) = val;
+    *reinterpret_cast<uint4*>(rowp + (u0 + 1) * 16) = val;
     fence_proxy_async_smem();
   }
-  if (warp == 0) tmem_alloc(tmem_slot, 512);
+  if (warp == 0) tmem_alloc(tmem_slot, C::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -236,12 +241,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t idesc_s = make_idesc_bf16(128, 128, false, false);          // S, dP
   const uint32_t idesc_dq = make_idesc_bf16(128, D, false, true);            // dS (K-major) x K (MN-major)
   const uint32_t idesc_dv = make_idesc_bf16(128, D, true, true);             // P^T (MN-major) x dO (MN-major)
-  const uint32_t idesc_dk = make_idesc_bf16(128, D + 64, true, true);        // dS^T x [Q | 1]
+  const uint32_t idesc_dk = make_idesc_bf16(128, D, true, true);            // dS^T x Q
+  const uint32_t idesc_ddt = make_idesc_bf16(128, 16, true, false);         // dS^T x ones (K-major)
   const uint32_t q_lo = desc_lo(smem_u32(sQ), 16), do_lo = desc_lo(smem_u32(sDO), 16);
-  const uint32_t qmn_lo = desc_lo(smem_u32(sQ), C::kSlabBytes);              // [Q | 1] as an MN-major B
+  const uint32_t qmn_lo = desc_lo(smem_u32(sQ), C::kSlabBytes);              // Q as an MN-major B
   const uint32_t domn_lo = desc_lo(smem_u32(sDO), C::kSlabBytes);
-  const uint32_t p_k_lo = desc_lo(smem_u32(sP), 16), ds_k_lo = desc_lo(smem_u32(sDS), 16);
-  const uint32_t p_mn_lo = desc_lo(smem_u32(sP), 16384), ds_mn_lo = desc_lo(smem_u32(sDS), 16384);
+  const uint32_t ones_lo = desc_lo(smem_u32(sOnes), 16);
+  const uint32_t ds_k_lo = desc_lo(smem_u32(sP), 16);                        // the buffer as a K-major A
+  const uint32_t p_mn_lo = desc_lo(smem_u32(sP), 16384);                    // ... and as an MN-major A (transposed)
 
   // S = X K_s^T (X = Q or dO, K-major both) into TMEM column col
   auto issue_xkt = [&](uint32_t x_lo, uint32_t k_lo, uint32_t col) {
@@ -313,19 +320,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                            : ((m == -INFINITY) ? 0.0f : m + log2f(l));
 
   // ---- pass 2: gradients ------------------------------------------------------
+  // per key tile: S = Q K^T; P (float32, kept in registers) stored as bf16;
+  // dP = dO V^T into the same TMEM columns with dV_t = P^T dO beside them;
+  // dS = P (dP - D) over P in shared memory; then dQ += dS K, dK_t = dS^T Q
+  // and d_dt = dS^T 1; thread r adds key r's dV, dK and d_dt to the
+  // accumulators
   if (ok && n_kt > 0) load_tile(0, gs % C::kStages, true);
   for (int j = 0; ok && j < n_kt; ++j, ++gs) {
     const int s = gs % C::kStages;
     ok = mbar_wait(kv_full + s, phase_kv[s] & 1, err, kDevErrTimeoutBase + 43);
     phase_kv[s] ^= 1u;
     __syncthreads();
-    if (C::kStages == 2 && j + 1 < n_kt) load_tile(j + 1, (gs + 1) % C::kStages, true);
     const uint32_t k_lo = desc_lo(smem_u32(sK + s * C::kKVBytes), 16);
     const uint32_t v_lo = desc_lo(smem_u32(sV + s * C::kKVBytes), 16);
     if (ok && tid == 0) {
       tc_fence_after();
       issue_xkt(q_lo, k_lo, 0);              // S
-      issue_xkt(do_lo, v_lo, C::kColDK);      // dP
       umma_commit(mma_done);
     }
     ok = __syncthreads_and(ok && wait_mma());
@@ -333,37 +343,64 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tc_fence_after();
     const float* mb = reinterpret_cast<const float*>(sMeta + s * C::kMetaBytes);
     const uint32_t* ms = reinterpret_cast<const uint32_t*>(mb + kKeyTile);
-    // P and dS of this row, 32 keys at a time, stored as bf16 [row][key] (128-byte swizzle)
-#pragma unroll
-    for (int c0 = 0; c0 < 128; c0 += 32) {
-      uint32_t rs[32], rp[32];
-      DMA_TMEM_LD32(tmem + lane_base + c0, rs);
-      DMA_TMEM_LD32(tmem + lane_base + C::kColDK + c0, rp);
-      tmem_wait_ld();
-      uint32_t pp[16], dd[16];
-#pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        float pv[2], dv[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const uint32_t sp = ms[c0 + c + e];
-          const bool kept = static_cast<uint32_t>(row - static_cast<int>(sp & 0xFFFFu)) < ((sp >> 16) - (sp & 0xFFFFu));
-          const float x = (__uint_as_float(rs[c + e]) * scale + mb[c0 + c + e]) * kLog2eB;
-          const float p = kept ? exp2f(x - lse) : 0.0f;
-          pv[e] = p;
-          dv[e] = p * (__uint_as_float(rp[c + e]) - Dr);
-        }
-        pp[c / 2] = pack_bf16x2(pv[0], pv[1]);
-        dd[c / 2] = pack_bf16x2(dv[0], dv[1]);
-      }
-      // keys c0 .. c0+31: chunk kc = c0 / 64, 16-byte units u0 .. u0+3
+    // P of this row, 32 keys at a time, kept in float32 and stored as bf16
+    // [row][key] (128-byte swizzle): keys c0 .. c0+31 are chunk c0 / 64, 16-byte units u0 .. u0+3
+    float pr[128];
+    auto store_row = [&](int c0, const uint32_t (&pk)[16]) {
       const int kc = c0 / 64, u0 = (c0 % 64) / 8;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const uint32_t off = kc * 16384 + row * 128 + ((((u0 + u) ^ (row & 7))) << 4);
-        *reinterpret_cast<uint4*>(sP + off) = make_uint4(pp[4 * u], pp[4 * u + 1], pp[4 * u + 2], pp[4 * u + 3]);
-        *reinterpret_cast<uint4*>(sDS + off) = make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
+        *reinterpret_cast<uint4*>(sP + off) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
       }
+    };
+#pragma unroll
+    for (int c0 = 0; c0 < 128; c0 += 32) {
+      uint32_t rs[32];
+      DMA_TMEM_LD32(tmem + lane_base + c0, rs);
+      tmem_wait_ld();
+      uint32_t pk[16];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const uint32_t sp = ms[c0 + c];
+        const bool kept = static_cast<uint32_t>(row - static_cast<int>(sp & 0xFFFFu)) < ((sp >> 16) - (sp & 0xFFFFu));
+        const float x = (__uint_as_float(rs[c]) * scale + mb[c0 + c]) * kLog2eB;
+        pr[c0 + c] = kept ? exp2f(x - lse) : 0.0f;
+      }
+#pragma unroll
+      for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(pr[c0 + 2 * c], pr[c0 + 2 * c + 1]);
+      store_row(c0, pk);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      issue_xkt(do_lo, v_lo, 0);             // dP over S's columns
+      // dV_t = P^T dO  (M = keys, K = rows: both operands MN-major)
+#pragma unroll
+      for (int kk = 0; kk < kRowTile / 16; ++kk) {
+        const uint32_t step = static_cast<uint32_t>((kk * 2048) >> 4);
+        if (kk == 0) umma_ss_w<0, kDescHiSw128, kDescHiSw128>(tmem + C::kColDV, p_mn_lo, domn_lo, idesc_dv);
+        else umma_ss_w<1, kDescHiSw128, kDescHiSw128>(tmem + C::kColDV, p_mn_lo + step, domn_lo + step, idesc_dv);
+      }
+      umma_commit(mma_done);
+    }
+    ok = __syncthreads_and(ok && wait_mma());
+    if (!ok) break;
+    tc_fence_after();
+    // dS = P (dP - D) over P in shared memory (dV_t, its reader, is done)
+#pragma unroll
+    for (int c0 = 0; c0 < 128; c0 += 32) {
+      uint32_t rp[32];
+      DMA_TMEM_LD32(tmem + lane_base + c0, rp);
+      tmem_wait_ld();
+      uint32_t dd[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        dd[c] = pack_bf16x2(pr[c0 + 2 * c] * (__uint_as_float(rp[2 * c]) - Dr),
+                            pr[c0 + 2 * c + 1] * (__uint_as_float(rp[2 * c + 1]) - Dr));
+      store_row(c0, dd);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -379,16 +416,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (kk == 0 && j == 0) umma_ss_w<0, kDescHiSw128, kDescHiSw128>(tmem + C::kColDQ, a, bb, idesc_dq);
         else umma_ss_w<1, kDescHiSw128, kDescHiSw128>(tmem + C::kColDQ, a, bb, idesc_dq);
       }
-      // dV_t = P^T dO and dK_t = dS^T [Q | 1]  (M = keys, K = rows: both operands MN-major)
+      // dK_t = dS^T Q and d_dt = dS^T 1  (M = keys, K = rows; dS^T is the MN-major view)
 #pragma unroll
       for (int kk = 0; kk < kRowTile / 16; ++kk) {
         const uint32_t step = static_cast<uint32_t>((kk * 2048) >> 4);
+        const uint32_t ostep = static_cast<uint32_t>(((kk / 4) * 2048 + (kk % 4) * 32) >> 4);
         if (kk == 0) {
-          umma_ss_w<0, kDescHiSw128, kDescHiSw128>(tmem, p_mn_lo, domn_lo, idesc_dv);
-          umma_ss_w<0, kDescHiSw128, kDescHiSw128>(tmem + C::kColDK, ds_mn_lo, qmn_lo, idesc_dk);
+          umma_ss_w<0, kDescHiSw128, kDescHiSw128>(tmem + C::kColDK, p_mn_lo, qmn_lo, idesc_dk);
+          umma_ss_w<0, kDescHiSw128, kDescHiSw128>(tmem + C::kColDDT, p_mn_lo, ones_lo, idesc_ddt);
         } else {
-          umma_ss_w<1, kDescHiSw128, kDescHiSw128>(tmem, p_mn_lo + step, domn_lo + step, idesc_dv);
-          umma_ss_w<1, kDescHiSw128, kDescHiSw128>(tmem + C::kColDK, ds_mn_lo + step, qmn_lo + step, idesc_dk);
+          umma_ss_w<1, kDescHiSw128, kDescHiSw128>(tmem + C::kColDK, p_mn_lo + step, qmn_lo + step, idesc_dk);
+          umma_ss_w<1, kDescHiSw128, kDescHiSw128>(tmem + C::kColDDT, p_mn_lo + step, ones_lo + ostep, idesc_ddt);
         }
       }
       umma_commit(mma_done);
@@ -405,7 +443,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t rv[32], rk[32];
-        DMA_TMEM_LD32(tmem + lane_base + c0, rv);
+        DMA_TMEM_LD32(tmem + lane_base + C::kColDV + c0, rv);
         DMA_TMEM_LD32(tmem + lane_base + C::kColDK + c0, rk);
         tmem_wait_ld();
         if (live) {
@@ -419,13 +457,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
       uint32_t rb[16];
-      DMA_TMEM_LD16(tmem + lane_base + C::kColDK + D, rb);
+      DMA_TMEM_LD16(tmem + lane_base + C::kColDDT, rb);
       tmem_wait_ld();
       if (live) atomicAdd(ddt32 + (static_cast<size_t>(b) * Hkv + g) * L + mk[tid], __uint_as_float(rb[0]));
     }
     tc_fence_before();
-    __syncthreads();   // TMEM, P, dS and the stage are free for the next tile
-    if (C::kStages == 1 && j + 1 < n_kt) load_tile(j + 1, (gs + 1) % C::kStages, true);
+    __syncthreads();   // TMEM, the P/dS buffer and the stage are free for the next tile
+    if (j + 1 < n_kt) load_tile(j + 1, (gs + 1) % C::kStages, true);
   }
 
   // dQ = scale * (dS K) summed over the list
@@ -451,7 +489,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, 512);
+  if (warp == 0) tmem_dealloc(tmem, C::kTmemCols);
 }
 
 // ---- the dt chain, one warp per token ------------------------------------------------

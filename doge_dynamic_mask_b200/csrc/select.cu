@@ -555,6 +555,34 @@ __device__ int sampled_collect(const uint32_t* __restrict__ bits, int n, int w, 
   return row_collect_ge_regions(bits, n, t_lo, out, cap, sc.red);
 }
 
+// A row tile that lies wholly past its sequence's last valid row: every row
+// sees the same keys and keeps K (w keys, sorted by key), so its tau is K's
+// smallest key and the list is K, each kept by every row.  Every thread must
+// call it.
+static __device__ __noinline__ void list_whole_set(const uint64_t* K, int w, int nrows, uint64_t* tau_rows,
+                                                   PrefillPlan plan, size_t tile) {
+  int32_t* idx_o = plan.idx + tile * plan.cap;
+  float* bias_o = plan.bias + tile * plan.cap;
+  uint32_t* span_o = plan.span + tile * plan.cap;
+  const uint64_t tau_last = K[w - 1];
+  for (int i = threadIdx.x; i < nrows; i += blockDim.x) tau_rows[i] = tau_last;
+  for (int e = threadIdx.x; e < w; e += blockDim.x) {
+    const uint64_t key = K[e];
+    idx_o[e] = static_cast<int32_t>(composite_index(key));
+    bias_o[e] = __uint_as_float(static_cast<uint32_t>(key >> 32));
+    span_o[e] = static_cast<uint32_t>(nrows) << 16;
+  }
+  const int padded = (w + kKeyTile - 1) / kKeyTile * kKeyTile;
+  for (int j = w + threadIdx.x; j < padded; j += blockDim.x) {
+    idx_o[j] = 0;
+    bias_o[j] = 0.0f;
+    span_o[j] = 0u;
+  }
+  int32_t* kb = plan.kbase + tile * (plan.cap / kKeyTile);
+  for (int kt = threadIdx.x; kt * kKeyTile < w; kt += blockDim.x) kb[kt] = -1;   // listed by key, not by index
+  if (threadIdx.x == 0) plan.counts[tile] = make_int2(w, w);
+}
+
 // One CTA per (batch, kv head, run of tpc consecutive row tiles).
 //
 // The CTA keeps the union U of a tile (the keys any of its rows keeps) sorted
@@ -644,6 +672,15 @@ __global__ void __launch_bounds__(kSelPrefillThreads, kSelPrefillMinBlocks) sele
     const int q_next = more ? min(r0 + kRowTile + min(kRowTile, L - r0 - kRowTile) - 1, len - 1) : q;
     uint32_t pre_next = 0u;
     if (more && tid < q_next - q) pre_next = __ldg(bits + q + 1 + tid);
+
+    if (have && p == q_prev) {
+      // the whole tile lies past the sequence's last valid row: every row
+      // keeps the carried K; K, cur and tau0 carry over unchanged
+      list_whole_set(Ubuf + static_cast<size_t>(cur) * ucap, w, nrows, tau_g + r0, plan, tile);
+      q_prev = q;
+      have = more;
+      continue;
+    }
 
     // K, the kept set at p (tau0 and above, at or before p), sorted, in buffer cur
     int n_keep, j_new;   // keys of K at or above tau0; the new keys are (j_new, q]

@@ -434,12 +434,16 @@ __global__ void __launch_bounds__(kBwdThreads, BwdCfg<D>::kMinBlocks)
     ok = __syncthreads_and(ok && wait_mma());
     if (!ok) break;
     tc_fence_after();
-    // thread = key of the tile: add its dV, dK and d_dt rows to the accumulators
+    // thread = key of the tile: add its dV, dK and d_dt rows to the accumulators.
+    // Every MMA of the tile is done, so the next tile's K, V and list metadata
+    // can load now, under the reductions (each thread first takes its own key
+    // index out of the metadata slot the load rewrites).
     {
       const int e = j * kKeyTile + tid;
-      const int32_t* mk = reinterpret_cast<const int32_t*>(ms + kKeyTile);
+      const int key = reinterpret_cast<const int32_t*>(ms + kKeyTile)[tid];
       const bool live = e < n_total;
-      const size_t krow = (static_cast<size_t>(base_row) + mk[tid]) * Hkv + g;
+      const size_t krow = (static_cast<size_t>(base_row) + key) * Hkv + g;
+      if (j + 1 < n_kt) load_tile(j + 1, (gs + 1) % C::kStages, true);
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t rv[32], rk[32];
@@ -459,11 +463,10 @@ __global__ void __launch_bounds__(kBwdThreads, BwdCfg<D>::kMinBlocks)
       uint32_t rb[16];
       DMA_TMEM_LD16(tmem + lane_base + C::kColDDT, rb);
       tmem_wait_ld();
-      if (live) atomicAdd(ddt32 + (static_cast<size_t>(b) * Hkv + g) * L + mk[tid], __uint_as_float(rb[0]));
+      if (live) atomicAdd(ddt32 + (static_cast<size_t>(b) * Hkv + g) * L + key, __uint_as_float(rb[0]));
     }
     tc_fence_before();
-    __syncthreads();   // TMEM, the P/dS buffer and the stage are free for the next tile
-    if (j + 1 < n_kt) load_tile(j + 1, (gs + 1) % C::kStages, true);
+    __syncthreads();   // TMEM and the P/dS buffer are free for the next tile
   }
 
   // dQ = scale * (dS K) summed over the list

@@ -21,6 +21,9 @@
 //     ascending run, else tile::gather4 (four listed rows per instruction).
 //     It also writes the tile's bias columns (below) and row intervals.
 //   * warp 2 (V producer): the same for V, on its own ring release.
+//   * warp 3 (gather helper, d = 128): a third of the four-row groups of
+//     every gathered K and V tile, since one warp issues its copies one at a
+//     time.
 //   * warp 1: allocates the 512 TMEM columns and, one thread, issues
 //     tcgen05.mma from 32-bit descriptor low words (the high words are
 //     constants).  S_h = Q_h K^T (M=128, N=128, K=d) plus one more K=16 step
@@ -56,7 +59,7 @@ namespace dma {
 namespace {
 
 // 12 warps in three warpgroups: warpgroup 0 = K producer, MMA issuer (and TMEM
-// owner), V producer and one spare warp; warpgroups 1 and 2 = the softmax of the
+// owner), V producer and gather helper; warpgroups 1 and 2 = the softmax of the
 // pair's two heads (four warps each, one per TMEM lane quarter).  The block is
 // launched with at most 168 registers per thread; warpgroup 0 then gives
 // registers back (setmaxnreg.dec) and the softmax warpgroups take them
@@ -73,6 +76,13 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units
 // (exp2_poly_x2), the rest on the MUFU
 constexpr int kPolyEvery = 5;
 constexpr int kXBytes = kKeyTile * 32;       // 128 rows x 16 bf16 extra K columns (bias / ones)
+// A gathered K or V tile is 32 groups of four listed rows, one tile::gather4
+// per group and 64-column slab.  A warp issues its lanes' copies one after
+// another (about 70 cycles each), so at d = 128 the copies of a tile are split
+// over three warps: the K and the V producer take groups [0, kGatherSplit) of
+// their tensor, the helper warp the remaining groups of both (44 / 44 / 40
+// copies per tile).
+constexpr int kGatherSplit = 22;
 
 template <int D>
 struct Cfg {
@@ -95,6 +105,10 @@ struct Cfg {
   // the softmax releases S as soon as it has read it, and the next S = Q K^T
   // overlaps the current softmax.  At d = 128 (O 2x128) P is written over S.
   static constexpr bool kSepP = D == 64;
+  // d = 128 splits its gathers over a third warp (kGatherSplit); at d = 64 a
+  // tile is half as many copies and the split measured slower, so the K and
+  // V producers issue all of theirs
+  static constexpr bool kHelper = D == 128;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;     // + alignment slack
   static constexpr uint32_t kTmemCols = 512;
@@ -295,8 +309,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bars.q_full, 1);
     mbar_init(bars.q_empty, 1);
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(bars.k_full + s, 1);
-      mbar_init(bars.v_full + s, 1);
+      // the producer's expect-tx arrival and the gather helper's arrival
+      mbar_init(bars.k_full + s, C::kHelper ? 2 : 1);
+      mbar_init(bars.v_full + s, C::kHelper ? 2 : 1);
       mbar_init(bars.k_empty + s, 1);
       mbar_init(bars.v_empty + s, 1);
     }
@@ -490,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_3d(sK + s * C::kKVBytes + sl * C::kSlabBytes, &tmap_k3, bars.k_full + s, sl * 64, g,
                           base_row + kb0);
           }
-        } else {
+        } else if (lane < (C::kHelper ? kGatherSplit : 32)) {
 #pragma unroll
           for (int sl = 0; sl < C::kSlabs; ++sl)
             tma_gather4(sK + s * C::kKVBytes + sl * C::kSlabBytes + lane * 512, &tmap_k, bars.k_full + s, sl * 64,
@@ -553,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_3d(sV + s * C::kKVBytes + sl * C::kSlabBytes, &tmap_v3, bars.v_full + s, sl * 64, g,
                           base_row + kb0);
           }
-        } else {
+        } else if (lane < (C::kHelper ? kGatherSplit : 32)) {
 #pragma unroll
           for (int sl = 0; sl < C::kSlabs; ++sl)
             tma_gather4(sV + s * C::kKVBytes + sl * C::kSlabBytes + lane * 512, &tmap_v, bars.v_full + s, sl * 64,
@@ -564,6 +579,74 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       for (int j = gv - C::kStages < 0 ? 0 : gv - C::kStages; j < gv; ++j)
         mbar_wait(bars.v_full + j % C::kStages, (j / C::kStages) & 1, err, kDevErrTimeoutBase + 3);
+    }
+  } else if (warp == 3 && C::kHelper) {
+    // ======================= K/V gather helper ==============================
+    // Row groups [kGatherSplit, 32) of every gathered K and V tile.  It arrives
+    // on every tile's full barriers (a run loaded as boxes included), so a
+    // full phase needs it and it can never fall two phases behind on the
+    // empty barriers it waits on.
+    const int rg = kGatherSplit + lane;
+    const bool active = rg < kKeyTile / 4;
+    int gh = 0;
+    bool stop = false;
+    ItemInfo x;
+    for (int i = 0; !stop && item_info(i, x); ++i) {
+      const int g = x.it.g, base_row = x.it.b * L;
+      const int32_t* idx_t = plan.idx + x.tile * plan.cap;
+      const int32_t* kbase_t = plan.kbase + x.tile * (plan.cap / kKeyTile);
+      auto fetch_kb = [&](int j) { return plan.no_topk ? j * kKeyTile : kbase_t[j]; };
+      auto fetch_ix = [&](int j) {
+        return plan.no_topk || !active ? make_int4(0, 0, 0, 0)
+                                       : *reinterpret_cast<const int4*>(idx_t + j * kKeyTile + rg * 4);
+      };
+      int nkb = x.n_kt > 0 ? fetch_kb(0) : 0;
+      int4 nix = x.n_kt > 0 ? fetch_ix(0) : make_int4(0, 0, 0, 0);
+      for (int j = 0; !stop && j < x.n_kt; ++j, ++gh) {
+        const int kb0 = nkb;
+        int4 ix = nix;
+        if (j + 1 < x.n_kt) {
+          nkb = fetch_kb(j + 1);
+          nix = fetch_ix(j + 1);
+        }
+        if (kb0 < 0) {
+          ix.x = (base_row + ix.x) * Hkv + g;
+          ix.y = (base_row + ix.y) * Hkv + g;
+          ix.z = (base_row + ix.z) * Hkv + g;
+          ix.w = (base_row + ix.w) * Hkv + g;
+        }
+        const int s = gh % C::kStages;
+        const int u = gh / C::kStages;
+        for (int kv = 0; kv < 2; ++kv) {
+          uint64_t* empty = (kv == 0 ? bars.k_empty : bars.v_empty) + s;
+          uint64_t* full = (kv == 0 ? bars.k_full : bars.v_full) + s;
+          if (gh >= C::kStages && !mbar_wait(empty, (u - 1) & 1, err, kDevErrTimeoutBase + 16 + kv)) {
+            *abort_flag = 1;
+            stop = true;
+            break;
+          }
+          if (aborted(abort_flag)) {
+            stop = true;
+            break;
+          }
+          if (kb0 < 0 && active) {
+            unsigned char* dst = (kv == 0 ? sK : sV) + s * C::kKVBytes + rg * 512;
+            const CUtensorMap* tm = kv == 0 ? &tmap_k : &tmap_v;
+#pragma unroll
+            for (int sl = 0; sl < C::kSlabs; ++sl)
+              tma_gather4(dst + sl * C::kSlabBytes, tm, full, sl * 64, ix.x, ix.y, ix.z, ix.w);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(full);
+        }
+      }
+    }
+    // drain: this warp's copies must have landed before the CTA can leave
+    if (lane == 0) {
+      for (int j = gh - C::kStages < 0 ? 0 : gh - C::kStages; j < gh; ++j) {
+        mbar_wait(bars.k_full + j % C::kStages, (j / C::kStages) & 1, err, kDevErrTimeoutBase + 18);
+        mbar_wait(bars.v_full + j % C::kStages, (j / C::kStages) & 1, err, kDevErrTimeoutBase + 18);
+      }
     }
   } else if (warp == 1) {
     // ======================= MMA issuer =====================================

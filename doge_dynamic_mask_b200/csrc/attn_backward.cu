@@ -76,6 +76,12 @@ struct BwdCfg {
   static_assert(D != 64 || 2 * (kSmemBytes + 1024) <= 233472, "two CTAs per SM at d = 64");
 };
 
+__device__ __forceinline__ unsigned long long mul_f32x2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 __device__ __forceinline__ float ld_bf16(const uint16_t* p) { return __uint_as_float(static_cast<uint32_t>(*p) << 16); }
 
 // red.global.add on four consecutive floats (16-byte aligned)
@@ -158,6 +164,7 @@ __global__ void __launch_bounds__(kBwdThreads, BwdCfg<D>::kMinBlocks)
   // counts come from it (the selector)
   pdl_wait();
   const int2 cnt = plan.counts[tile];
+  const int n_full = cnt.x;   // list entries below n_full are kept by every row of the tile
   const int n_total = cnt.y;
   const int n_kt = (n_total + kKeyTile - 1) / kKeyTile;
 
@@ -354,6 +361,14 @@ __global__ void __launch_bounds__(kBwdThreads, BwdCfg<D>::kMinBlocks)
         *reinterpret_cast<uint4*>(sP + off) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
       }
     };
+    // x = log2e (scale q.k + bias) - lse as one FMA per key: scale log2e is a
+    // constant, log2e bias - lse comes from the key's bias; on a key tile kept
+    // by every row the row intervals need no check (rows past the sequence
+    // still get P = 0)
+    const bool full_tile = (j + 1) * kKeyTile <= n_full;
+    const float sl2e = scale * kLog2eB;
+    const float4* mb4 = reinterpret_cast<const float4*>(mb);
+    const uint4* ms4 = reinterpret_cast<const uint4*>(ms);
 #pragma unroll
     for (int c0 = 0; c0 < 128; c0 += 32) {
       uint32_t rs[32];
@@ -361,11 +376,23 @@ __global__ void __launch_bounds__(kBwdThreads, BwdCfg<D>::kMinBlocks)
       tmem_wait_ld();
       uint32_t pk[16];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const uint32_t sp = ms[c0 + c];
-        const bool kept = static_cast<uint32_t>(row - static_cast<int>(sp & 0xFFFFu)) < ((sp >> 16) - (sp & 0xFFFFu));
-        const float x = (__uint_as_float(rs[c]) * scale + mb[c0 + c]) * kLog2eB;
-        pr[c0 + c] = kept ? exp2f(x - lse) : 0.0f;
+      for (int c4 = 0; c4 < 8; ++c4) {
+        const float4 bb = mb4[c0 / 4 + c4];
+        const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+        uint32_t spv[4] = {0u, 0u, 0u, 0u};
+        if (!full_tile) {
+          const uint4 sp4 = ms4[c0 / 4 + c4];
+          spv[0] = sp4.x; spv[1] = sp4.y; spv[2] = sp4.z; spv[3] = sp4.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = 4 * c4 + e;
+          const bool kept = full_tile ? row_valid
+                                      : static_cast<uint32_t>(row - static_cast<int>(spv[e] & 0xFFFFu)) <
+                                            ((spv[e] >> 16) - (spv[e] & 0xFFFFu));
+          const float x = fmaf(__uint_as_float(rs[c]), sl2e, fmaf(bv[e], kLog2eB, -lse));
+          pr[c0 + c] = kept ? fast_exp2(x) : 0.0f;
+        }
       }
 #pragma unroll
       for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(pr[c0 + 2 * c], pr[c0 + 2 * c + 1]);
@@ -396,10 +423,16 @@ __global__ void __launch_bounds__(kBwdThreads, BwdCfg<D>::kMinBlocks)
       DMA_TMEM_LD32(tmem + lane_base + c0, rp);
       tmem_wait_ld();
       uint32_t dd[16];
+      const unsigned long long dr2 = f32x2(Dr, Dr);
 #pragma unroll
-      for (int c = 0; c < 16; ++c)
-        dd[c] = pack_bf16x2(pr[c0 + 2 * c] * (__uint_as_float(rp[2 * c]) - Dr),
-                            pr[c0 + 2 * c + 1] * (__uint_as_float(rp[2 * c + 1]) - Dr));
+      for (int c = 0; c < 16; ++c) {
+        const unsigned long long ds2 =
+            mul_f32x2(f32x2(pr[c0 + 2 * c], pr[c0 + 2 * c + 1]),
+                      sub_f32x2(f32x2(__uint_as_float(rp[2 * c]), __uint_as_float(rp[2 * c + 1])), dr2));
+        float d0, d1;
+        f32x2_split(ds2, d0, d1);
+        dd[c] = pack_bf16x2(d0, d1);
+      }
       store_row(c0, dd);
     }
     fence_proxy_async_smem();

@@ -84,6 +84,18 @@ __device__ __forceinline__ unsigned long long mul_f32x2(unsigned long long a, un
 
 __device__ __forceinline__ float ld_bf16(const uint16_t* p) { return __uint_as_float(static_cast<uint32_t>(*p) << 16); }
 
+// TMA reduce-add of a shared-memory box into a 3-D float32 tensor map
+// (bulk async-group completion)
+__device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, const void* src, int c0, int c1, int c2) {
+  asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // red.global.add on four consecutive floats (16-byte aligned)
 __device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
@@ -95,6 +107,7 @@ __global__ void __launch_bounds__(kBwdThreads, BwdCfg<D>::kMinBlocks)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_do,
                     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                     const __grid_constant__ CUtensorMap tmap_k3, const __grid_constant__ CUtensorMap tmap_v3,
+                    const __grid_constant__ CUtensorMap tmap_dk, const __grid_constant__ CUtensorMap tmap_dv,
                     PrefillPlan plan, int B, int L, int Hq, int Hkv, float scale, const uint16_t* __restrict__ out,
                     const uint16_t* __restrict__ dout, const float* __restrict__ lse_in, uint16_t* __restrict__ dq,
                     float* __restrict__ dk32, float* __restrict__ dv32, float* __restrict__ ddt32, uint32_t* err) {
@@ -477,19 +490,57 @@ __global__ void __launch_bounds__(kBwdThreads, BwdCfg<D>::kMinBlocks)
       const bool live = e < n_total;
       const size_t krow = (static_cast<size_t>(base_row) + key) * Hkv + g;
       if (j + 1 < n_kt) load_tile(j + 1, (gs + 1) % C::kStages, true);
+      const int kb0 = kbase_t[j];
+      if (kb0 >= 0) {
+        // the tile's keys are the run kb0 .. kb0 + 127: 64 columns of dV, then
+        // of dK, at a time are staged in the P/dS buffer (free now; two boxes
+        // of 32 float32 columns, 128-byte swizzle) and TMA adds them into the
+        // accumulators.  Rows of list padding are zero (P = 0 there).
+#pragma unroll 1
+        for (int rnd = 0; rnd < 2 * (D / 64); ++rnd) {
+          const bool is_k = rnd >= D / 64;
+          const int col0 = (rnd % (D / 64)) * 64;
+          const uint32_t tcol = (is_k ? C::kColDK : C::kColDV) + col0;
+          const float mul = is_k ? scale : 1.0f;
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t rv[32], rk[32];
-        DMA_TMEM_LD32(tmem + lane_base + C::kColDV + c0, rv);
-        DMA_TMEM_LD32(tmem + lane_base + C::kColDK + c0, rk);
-        tmem_wait_ld();
-        if (live) {
+          for (int bx = 0; bx < 2; ++bx) {
+            uint32_t r[32];
+            DMA_TMEM_LD32(tmem + lane_base + tcol + 32 * bx, r);
+            tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; c += 4) {
-            red_add_v4(dv32 + krow * D + c0 + c, __uint_as_float(rv[c]), __uint_as_float(rv[c + 1]),
-                       __uint_as_float(rv[c + 2]), __uint_as_float(rv[c + 3]));
-            red_add_v4(dk32 + krow * D + c0 + c, __uint_as_float(rk[c]) * scale, __uint_as_float(rk[c + 1]) * scale,
-                       __uint_as_float(rk[c + 2]) * scale, __uint_as_float(rk[c + 3]) * scale);
+            for (int ch = 0; ch < 8; ++ch) {
+              const uint32_t off = bx * 16384 + row * 128 + ((ch ^ (row & 7)) << 4);
+              *reinterpret_cast<float4*>(sP + off) =
+                  make_float4(__uint_as_float(r[4 * ch]) * mul, __uint_as_float(r[4 * ch + 1]) * mul,
+                              __uint_as_float(r[4 * ch + 2]) * mul, __uint_as_float(r[4 * ch + 3]) * mul);
+            }
+          }
+          fence_proxy_async_smem();
+          __syncthreads();
+          if (tid == 0) {
+#pragma unroll
+            for (int bx = 0; bx < 2; ++bx)
+              tma_reduce_add_3d(is_k ? &tmap_dk : &tmap_dv, sP + bx * 16384, col0 + 32 * bx, g, base_row + kb0);
+            bulk_commit();
+            bulk_wait_read_all();   // the buffer may be rewritten after the barrier
+          }
+          __syncthreads();
+        }
+      } else {
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t rv[32], rk[32];
+          DMA_TMEM_LD32(tmem + lane_base + C::kColDV + c0, rv);
+          DMA_TMEM_LD32(tmem + lane_base + C::kColDK + c0, rk);
+          tmem_wait_ld();
+          if (live) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 4) {
+              red_add_v4(dv32 + krow * D + c0 + c, __uint_as_float(rv[c]), __uint_as_float(rv[c + 1]),
+                         __uint_as_float(rv[c + 2]), __uint_as_float(rv[c + 3]));
+              red_add_v4(dk32 + krow * D + c0 + c, __uint_as_float(rk[c]) * scale, __uint_as_float(rk[c + 1]) * scale,
+                         __uint_as_float(rk[c + 2]) * scale, __uint_as_float(rk[c + 3]) * scale);
+            }
           }
         }
       }
@@ -522,6 +573,7 @@ __global__ void __launch_bounds__(kBwdThreads, BwdCfg<D>::kMinBlocks)
       }
     }
   }
+  if (tid == 0) bulk_wait_all();   // every TMA reduction has been applied
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -651,12 +703,27 @@ cudaError_t launch_bwd_d(const void* q, const void* k, const void* v, const void
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
+  // the float32 accumulators [B*L, Hkv, d] as TMA reduce-add targets: boxes of
+  // 32 columns x 128 consecutive keys of one kv head
+  CUtensorMap tdk, tdv;
+  float* acc[2] = {dk32, dv32};
+  CUtensorMap* amaps[2] = {&tdk, &tdv};
+  for (int i = 0; i < 2; ++i) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(g.Hkv), BL};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(g.Hkv) * D * 4};
+    cuuint32_t box[3] = {32, 1, static_cast<cuuint32_t>(kKeyTile)};
+    cuuint32_t es[3] = {1, 1, 1};
+    if (enc(amaps[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, acc[i], dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(attn_bwd_kernel<D>), C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const long long n_cta = static_cast<long long>(plan.n_row_tiles) * g.B * g.Hq;
   if (n_cta > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
   return launch_after(attn_bwd_kernel<D>, dim3(static_cast<unsigned>(n_cta)), dim3(kBwdThreads), C::kSmemBytes, s, tq,
-                      tdo, tk, tv, tk3, tv3, plan, g.B, g.Lk, g.Hq, g.Hkv, scale, static_cast<const uint16_t*>(out),
+                      tdo, tk, tv, tk3, tv3, tdk, tdv, plan, g.B, g.Lk, g.Hq, g.Hkv, scale, static_cast<const uint16_t*>(out),
                       static_cast<const uint16_t*>(dout), lse_in, static_cast<uint16_t*>(dq), dk32, dv32, ddt32, err);
 }
 

@@ -94,6 +94,7 @@ __device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, const void* 
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // red.global.add on four consecutive floats (16-byte aligned)
@@ -357,6 +358,7 @@ __global__ void __launch_bounds__(kBwdThreads, BwdCfg<D>::kMinBlocks)
       tc_fence_after();
       issue_xkt(q_lo, k_lo, 0);              // S
       umma_commit(mma_done);
+      bulk_wait_read_all();   // the previous tile's staged dV / dK boxes have been read
     }
     ok = __syncthreads_and(ok && wait_mma());
     if (!ok) break;
@@ -492,40 +494,38 @@ __global__ void __launch_bounds__(kBwdThreads, BwdCfg<D>::kMinBlocks)
       if (j + 1 < n_kt) load_tile(j + 1, (gs + 1) % C::kStages, true);
       const int kb0 = kbase_t[j];
       if (kb0 >= 0) {
-        // the tile's keys are the run kb0 .. kb0 + 127: 64 columns of dV, then
-        // of dK, at a time are staged in the P/dS buffer (free now; two boxes
-        // of 32 float32 columns, 128-byte swizzle) and TMA adds them into the
-        // accumulators.  Rows of list padding are zero (P = 0 there).
+        // the tile's keys are the run kb0 .. kb0 + 127: 32 columns of dV, then
+        // of dK, at a time (one box, 128-byte swizzle) are staged in one half
+        // of the P/dS buffer (free now) and TMA adds them into the
+        // accumulators; the halves alternate, so a box's read overlaps the
+        // staging of the next.  Rows of list padding are zero (P = 0 there).
+        constexpr int kRounds = 2 * (D / 32);
 #pragma unroll 1
-        for (int rnd = 0; rnd < 2 * (D / 64); ++rnd) {
-          const bool is_k = rnd >= D / 64;
-          const int col0 = (rnd % (D / 64)) * 64;
-          const uint32_t tcol = (is_k ? C::kColDK : C::kColDV) + col0;
+        for (int rnd = 0; rnd < kRounds; ++rnd) {
+          const bool is_k = rnd >= D / 32;
+          const int col0 = (rnd % (D / 32)) * 32;
           const float mul = is_k ? scale : 1.0f;
+          unsigned char* buf = sP + (rnd & 1) * 16384;
+          uint32_t r[32];
+          DMA_TMEM_LD32(tmem + lane_base + (is_k ? C::kColDK : C::kColDV) + col0, r);
+          tmem_wait_ld();
 #pragma unroll
-          for (int bx = 0; bx < 2; ++bx) {
-            uint32_t r[32];
-            DMA_TMEM_LD32(tmem + lane_base + tcol + 32 * bx, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-              const uint32_t off = bx * 16384 + row * 128 + ((ch ^ (row & 7)) << 4);
-              *reinterpret_cast<float4*>(sP + off) =
-                  make_float4(__uint_as_float(r[4 * ch]) * mul, __uint_as_float(r[4 * ch + 1]) * mul,
-                              __uint_as_float(r[4 * ch + 2]) * mul, __uint_as_float(r[4 * ch + 3]) * mul);
-            }
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint32_t off = row * 128 + ((ch ^ (row & 7)) << 4);
+            *reinterpret_cast<float4*>(buf + off) =
+                make_float4(__uint_as_float(r[4 * ch]) * mul, __uint_as_float(r[4 * ch + 1]) * mul,
+                            __uint_as_float(r[4 * ch + 2]) * mul, __uint_as_float(r[4 * ch + 3]) * mul);
           }
           fence_proxy_async_smem();
           __syncthreads();
           if (tid == 0) {
-#pragma unroll
-            for (int bx = 0; bx < 2; ++bx)
-              tma_reduce_add_3d(is_k ? &tmap_dk : &tmap_dv, sP + bx * 16384, col0 + 32 * bx, g, base_row + kb0);
+            tma_reduce_add_3d(is_k ? &tmap_dk : &tmap_dv, buf, col0, g, base_row + kb0);
             bulk_commit();
-            bulk_wait_read_all();   // the buffer may be rewritten after the barrier
+            bulk_wait_read_1();   // the other half (the previous box) has been read
           }
-          __syncthreads();
+          if (rnd + 1 < kRounds) __syncthreads();
         }
+        // the last box is read before the next tile writes P (thread 0 waits there)
       } else {
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {

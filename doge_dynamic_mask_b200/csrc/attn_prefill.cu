@@ -83,6 +83,10 @@ constexpr int kXBytes = kKeyTile * 32;       // 128 rows x 16 bf16 extra K colum
 // their tensor, the helper warp the remaining groups of both (44 / 44 / 40
 // copies per tile).
 constexpr int kGatherSplit = 22;
+// At d = 128 work items reach a CTA through a global counter (heaviest
+// first), fetched by the K producer and handed to the other roles through a
+// ring of kItemRing slots in shared memory.
+constexpr int kItemRing = 8;
 
 template <int D>
 struct Cfg {
@@ -100,7 +104,7 @@ struct Cfg {
   static constexpr int kOffV = kOffKx + kStages * kXBytes;
   static constexpr int kOffMeta = kOffV + kStages * kKVBytes;
   static constexpr int kOffBar = kOffMeta + kMetaSlots * kMetaBytes;
-  static constexpr int kNumBars = 2 + 4 * kStages + kMetaSlots + 8 + 1;
+  static constexpr int kNumBars = 2 + 4 * kStages + kMetaSlots + 8 + 1 + 2 * kItemRing;
   // d = 64 leaves TMEM room for P in its own columns (S 2x128, O 2x64, P 2x64):
   // the softmax releases S as soon as it has read it, and the next S = Q K^T
   // overlaps the current softmax.  At d = 128 (O 2x128) P is written over S.
@@ -109,8 +113,13 @@ struct Cfg {
   // tile is half as many copies and the split measured slower, so the K and
   // V producers issue all of theirs
   static constexpr bool kHelper = D == 128;
+  // d = 128 draws its work items from a global counter (their costs vary with
+  // the kept-key unions, ~14 items per CTA on long context); at d = 64 the
+  // static order measured faster (fewer, more even items per CTA)
+  static constexpr bool kDynamic = D == 128;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;     // + alignment slack
+  static constexpr int kOffRing = kOffMisc + 64;              // kItemRing work-item numbers
+  static constexpr int kSmemBytes = kOffRing + kItemRing * 4 + 1024;   // + alignment slack
   static constexpr uint32_t kTmemCols = 512;
   static_assert(2 * 128 + 2 * D <= 512, "TMEM budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -135,6 +144,8 @@ struct Bars {
   uint64_t* p_ready;    // [2]
   uint64_t* o_done;     // [2]
   uint64_t* fin;
+  uint64_t* item_full;    // [kItemRing] the slot holds the next work item's number
+  uint64_t* item_empty;   // [kItemRing] every other role has read the slot
 };
 
 __device__ __forceinline__ bool aborted(volatile int* flag) { return *flag != 0; }
@@ -245,9 +256,10 @@ __device__ __forceinline__ Item decode_item(int w, int npairs, int Hkv, int B, i
   it.t = n_rt - 1 - w / B;
   return it;
 }
-// The i-th work item of this CTA: rounds of gridDim.x items, taken forwards in
-// even rounds and backwards in odd ones, so every CTA gets a similar mix of
-// heavy and light row tiles.
+
+// The i-th work item of this CTA in the static order: rounds of gridDim.x
+// items, taken forwards in even rounds and backwards in odd ones, so every CTA
+// gets a similar mix of heavy and light row tiles.
 __device__ __forceinline__ int item_of(int i) {
   const int P = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
   return i * P + ((i & 1) ? P - 1 - c : c);
@@ -283,7 +295,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bars.s_free = p; p += 2;
     bars.p_ready = p; p += 2;
     bars.o_done = p; p += 2;
-    bars.fin = p;
+    bars.fin = p; p += 1;
+    bars.item_full = p; p += kItemRing;
+    bars.item_empty = p;
   }
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
@@ -325,6 +339,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bars.o_done + h, 1);
     }
     mbar_init(bars.fin, 1);
+    for (int r = 0; r < kItemRing; ++r) {
+      mbar_init(bars.item_full + r, 1);
+      // V producer, MMA issuer, gather helper (d = 128) and the eight softmax warps
+      mbar_init(bars.item_empty + r, 2 + (C::kHelper ? 1 : 0) + 8);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -362,8 +381,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     int nh, n_kt, n_full, n_total;
     size_t tile;
   };
+  // The i-th work item of this CTA.  d = 64: the static order (item_of).
+  // d = 128: item 0 is blockIdx.x; later ones come
+  // from the counter (offset by the grid), heaviest first, so CTAs that drew
+  // light items take more.  The K producer fetches (one item ahead, so the
+  // atomic's latency is hidden) and publishes each number in ring slot
+  // i % kItemRing; the other roles wait for the slot, read it and release it.
+  // The last CTA to finish resets the counter (the workspace starts zeroed).
+  uint32_t* sched = err + 16;        // items handed out beyond the first wave
+  uint32_t* sched_done = err + 17;   // CTAs finished
+  int* ring = reinterpret_cast<int*>(smem + C::kOffRing);
+  int next_w = 0;                    // the K producer's prefetched number
+  auto fetch_item = [&](int i) -> int {
+    if constexpr (!C::kDynamic) return item_of(i);
+    const int slot = i % kItemRing;
+    const int lane_ = threadIdx.x & 31;
+    if (warp == 0) {
+      int wv = 0;
+      if (lane_ == 0) {
+        if (i == 0) {
+          wv = static_cast<int>(blockIdx.x);
+        } else {
+          wv = next_w;
+        }
+        next_w = static_cast<int>(atomicAdd(sched, 1u)) + static_cast<int>(gridDim.x);
+        if (i >= kItemRing &&
+            !mbar_wait(bars.item_empty + slot, ((i / kItemRing) - 1) & 1, err, kDevErrTimeoutBase + 23)) {
+          *abort_flag = 1;
+          wv = n_items;   // stop
+        }
+        ring[slot] = wv;
+        mbar_arrive(bars.item_full + slot);
+      }
+      return __shfl_sync(0xFFFFFFFFu, wv, 0);
+    }
+    int wv = n_items;   // stop on a wait that gives up
+    if (mbar_wait(bars.item_full + slot, (i / kItemRing) & 1, err, kDevErrTimeoutBase + 24)) wv = ring[slot];
+    else *abort_flag = 1;
+    if (warp == 1) {
+      mbar_arrive(bars.item_empty + slot);   // the issuing thread alone runs its loop
+    } else {
+      __syncwarp();
+      if (lane_ == 0) mbar_arrive(bars.item_empty + slot);
+    }
+    return wv;
+  };
   auto item_info = [&](int i, ItemInfo& x) -> bool {
-    const int w = item_of(i);
+    const int w = fetch_item(i);
     if (w >= n_items) return false;
     x.it = decode_item(w, npairs, Hkv, B, n_rt);
     x.nh = min(2, nrep - 2 * x.it.pair);
@@ -989,6 +1053,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
+  if (C::kDynamic && threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(sched_done, 1u) == gridDim.x - 1) {
+      // every CTA has drawn its last number: the next launch starts from zero
+      *sched = 0u;
+      *sched_done = 0u;
+      __threadfence();
+    }
+  }
 }
 
 // ---- host: tensor maps -------------------------------------------------------

@@ -188,6 +188,32 @@ def test_prefill_parity(dma, w_):
     assert_out_close(got2, want, "full path")
 
 
+@pytest.mark.parametrize("w_", [wl(2, 1500, 8, 2, 128, 300, lens=(700, 1500), seed=31),
+                                 wl(1, 640, 4, 4, 128, 700, seed=32)],
+                         ids=["topk_d128", "dense_d128"])
+def test_prefill_repeated_calls_share_a_workspace(dma, w_):
+    """At d = 128 the attention CTAs draw their work items from a counter in
+    the workspace header, which the last CTA resets: repeated calls on one
+    workspace must each cover every item exactly once (same bits every time,
+    matching the oracle) and leave the counter words at zero."""
+    dev, cpu = inputs(w_)
+    q, k, v = f64(cpu["q"]), f64(cpu["k"]), f64(cpu["v"])
+    W, A = cpu["W"].double().numpy(), cpu["A"].double().numpy()
+    dt32 = oracle.dt_scores(v, W, A)
+    want = oracle.prefill(q, k, v, None, None, cpu["lengths"].numpy(), w_.w, w_.scale, dt=dt32)
+    ws = dma.new_workspace(dma.dma_workspace_size(w_.B, w_.L, w_.L, w_.Hq, w_.Hkv, w_.d, w_.w))
+    outs = []
+    for _ in range(3):
+        outs.append(dma.dma_forward_prefill(dev["q"], dev["k"], dev["v"], dev["W"], dev["A"], dev["lengths"], w_.w,
+                                            workspace=ws).clone())
+        assert dma.dma_check(ws) == 0
+        header = ws[:256].view(torch.int32).cpu()
+        assert int(header[16]) == 0 and int(header[17]) == 0, "work-item counter not reset"
+    assert_out_close(outs[0], want, "first call")
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0]), "a repeated call differs"
+
+
 # ----------------------------------------------------------------------------
 # S4 decode
 # ----------------------------------------------------------------------------

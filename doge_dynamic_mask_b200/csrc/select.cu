@@ -614,7 +614,11 @@ __global__ void __launch_bounds__(kSelPrefillThreads, kSelPrefillMinBlocks) sele
   uint64_t* Ubuf = reinterpret_cast<uint64_t*>(smem_raw + sizeof(PrefillSelSmem));   // two buffers of ucap keys
   SelScratch sc{sm.hist, Ubuf, sm.red, sm.vars};   // the candidate buffer is dead before Ubuf is written
 
-  const int g = blockIdx.y, b = blockIdx.z;
+  // grid (kv head, batch, run): blocks start in that order, so the runs are
+  // taken from the end of the sequence backwards (the late runs, whose first
+  // tile selects over the longest prefix, start in the first wave)
+  const int g = blockIdx.x, b = blockIdx.y;
+  const int run = static_cast<int>(gridDim.z - 1 - blockIdx.z);
   const int len = clamp_len(lengths, b, L, err);
   const bool topk = L > w;
   const size_t bg = static_cast<size_t>(b) * Hkv + g;
@@ -623,7 +627,7 @@ __global__ void __launch_bounds__(kSelPrefillThreads, kSelPrefillMinBlocks) sele
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nw = static_cast<int>(blockDim.x >> 5);
   const uint32_t lt = lanemask_lt();
-  const int t_first = blockIdx.x * tpc;
+  const int t_first = run * tpc;
   const int t_last = min(plan.n_row_tiles, t_first + tpc);
   bool have = false;      // K(q') of the previous tile and this tile's tau0 carry over
   int cur = 0;            // buffer whose head holds K
@@ -1109,7 +1113,7 @@ cudaError_t launch_select_prefill(const float* dt, const int32_t* lengths, const
   const long long slots = static_cast<long long>(kSelPrefillMinBlocks) * nsm;
   long long tpc = (topk_tiles + slots - 1) / slots;
   tpc = tpc < 1 ? 1 : (tpc > kSelTilesPerCtaMax ? kSelTilesPerCtaMax : tpc);
-  dim3 grid(static_cast<unsigned>((plan.n_row_tiles + tpc - 1) / tpc), g.Hkv, g.B);
+  dim3 grid(g.Hkv, g.B, static_cast<unsigned>((plan.n_row_tiles + tpc - 1) / tpc));
   return launch_after(select_prefill_kernel, grid, dim3(kSelPrefillThreads), smem, s, dt, lengths, g.Hkv, L, g.w,
                       static_cast<int>(tpc), plan, err);
 }

@@ -194,8 +194,11 @@ def test_prefill_parity(dma, w_):
 def test_prefill_repeated_calls_share_a_workspace(dma, w_):
     """At d = 128 the attention CTAs draw their work items from a counter in
     the workspace header, which the last CTA resets: repeated calls on one
-    workspace must each cover every item exactly once (same bits every time,
-    matching the oracle) and leave the counter words at zero."""
+    workspace must each cover every item exactly once (each matches the
+    oracle) and leave the counter words at zero.  Without a top-k the lists
+    are built in key order, so the calls agree bit for bit; with one, the
+    order inside a list class is free (warps reserve their segments), so the
+    float32 sums may round differently from call to call."""
     dev, cpu = inputs(w_)
     q, k, v = f64(cpu["q"]), f64(cpu["k"]), f64(cpu["v"])
     W, A = cpu["W"].double().numpy(), cpu["A"].double().numpy()
@@ -209,9 +212,11 @@ def test_prefill_repeated_calls_share_a_workspace(dma, w_):
         assert dma.dma_check(ws) == 0
         header = ws[:256].view(torch.int32).cpu()
         assert int(header[16]) == 0 and int(header[17]) == 0, "work-item counter not reset"
-    assert_out_close(outs[0], want, "first call")
-    for o in outs[1:]:
-        assert torch.equal(o, outs[0]), "a repeated call differs"
+    for i, o in enumerate(outs):
+        assert_out_close(o, want, f"call {i}")
+    if w_.w >= w_.L:
+        for o in outs[1:]:
+            assert torch.equal(o, outs[0]), "a repeated call differs"
 
 
 # ----------------------------------------------------------------------------

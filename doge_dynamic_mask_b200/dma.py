@@ -274,11 +274,16 @@ def dma_decode_step_cached(q, k_cache, v_cache, W_dt, A, lengths, keep_window_si
     return out
 
 
+# keys per split of the decode attention: the kept lists are padded to a
+# multiple of it (the library's layout of a decode workspace)
+DECODE_CHUNK = 128
+
+
 def decode_state_views(state, B, Lk, Hq, Hkv, d, keep_window_size):
     """(dt [B, Hkv, Lk] float32, kept count [B, Hkv] int32, kept key lists [B, Hkv, cap] int32) views of a
     decode state, for tests: the layout is that of a decode workspace."""
     bg = B * Hkv
-    cap = -(-min(Lk, keep_window_size) // 128) * 128
+    cap = -(-min(Lk, keep_window_size) // DECODE_CHUNK) * DECODE_CHUNK
     def up(x):
         return -(-x // 256) * 256
     off = 256

@@ -123,15 +123,18 @@ __global__ void __launch_bounds__(kBwdThreads, BwdCfg<D>::kMinBlocks)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 4);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // work item: (b, g, t, head r of the group)
+  // work item: (b, g, t, head r of the group), the row tile slowest and the
+  // last (heaviest: the longest causal list) first, so the long CTAs start in
+  // the first waves and the light ones fill the end
   const int nrep = Hq / Hkv;
   int w = blockIdx.x;
   const int r_in_group = w % nrep;
   w /= nrep;
-  const int t = w % plan.n_row_tiles;
-  w /= plan.n_row_tiles;
   const int g = w % Hkv;
-  const int b = w / Hkv;
+  w /= Hkv;
+  const int b = w % B;
+  w /= B;
+  const int t = plan.n_row_tiles - 1 - w;
   const int h = g * nrep + r_in_group;
   const size_t tile = (static_cast<size_t>(b) * Hkv + g) * plan.n_row_tiles + t;
   const int r0 = t * kRowTile;

@@ -221,15 +221,9 @@ struct RouteSmem {
   float mout;                           // best pair score outside the candidate region
 };
 
-__device__ __forceinline__ float dot_bf16x8(uint4 a, uint4 b) {
-  const uint32_t x[4] = {a.x, a.y, a.z, a.w}, y[4] = {b.x, b.y, b.z, b.w};
-  float s = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    s = fmaf(__uint_as_float(x[i] << 16), __uint_as_float(y[i] << 16), s);
-    s = fmaf(__uint_as_float(x[i] & 0xFFFF0000u), __uint_as_float(y[i] & 0xFFFF0000u), s);
-  }
-  return s;
+// two bf16 channels (one 32-bit word, low channel first) as packed float32
+__device__ __forceinline__ unsigned long long widen_bf16x2(uint32_t w) {
+  return f32x2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
 // Keeps the k best of the domain's K <= blockDim keys, best first: thread j
@@ -340,6 +334,25 @@ __global__ void __launch_bounds__(kRouteThreads)
     if (threadIdx.x < k) sm.fin[rank] = mine;
     __syncthreads();
   }
+  // h of the token in float32, once, for the 64 down-row products: in the
+  // candidate-key buffer (free now) after the up-projection's partial sums
+  // (groups * hidden <= 8192 floats: hidden <= 8192, and groups * hidden =
+  // 8 * blockDim when a row has fewer pieces than the block has threads)
+  const int n16 = hidden / 8;   // 16-byte pieces per row
+  const int groups = n16 >= static_cast<int>(blockDim.x) ? 1 : static_cast<int>(blockDim.x) / n16;
+  float* hf = reinterpret_cast<float*>(sm.keys) + (groups - 1) * hidden;
+  {
+    const uint4* h4 = reinterpret_cast<const uint4*>(h + static_cast<size_t>(t) * hidden);
+    for (int c = threadIdx.x; c < n16; c += blockDim.x) {
+      const uint4 u = __ldg(h4 + c);
+      const uint32_t x[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        hf[8 * c + 2 * i] = __uint_as_float(x[i] << 16);
+        hf[8 * c + 2 * i + 1] = __uint_as_float(x[i] & 0xFFFF0000u);
+      }
+    }
+  }
   // 3. the kept experts and their scores, best first
   if (threadIdx.x < k) {
     const uint64_t mine = sm.fin[threadIdx.x];
@@ -354,14 +367,24 @@ __global__ void __launch_bounds__(kRouteThreads)
     experts_out[static_cast<size_t>(t) * k + threadIdx.x] = sm.ex[threadIdx.x];
     scores_out[static_cast<size_t>(t) * k + threadIdx.x] = sm.sc[threadIdx.x];
   }
-  // 4. down-projection: one warp per expert row, h . down_embed[e]
+  // 4. down-projection: one warp per expert row, h . down_embed[e] (packed
+  // float32 pairs against h in shared memory)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  const uint4* h4 = reinterpret_cast<const uint4*>(h + static_cast<size_t>(t) * hidden);
-  const int n16 = hidden / 8;   // 16-byte pieces per row
+  const float4* hf4 = reinterpret_cast<const float4*>(hf);
   for (int q = warp; q < k; q += nwarps) {
     const uint4* d4 = reinterpret_cast<const uint4*>(down_embed + static_cast<size_t>(sm.ex[q]) * hidden);
-    float acc = 0.0f;
-    for (int c = lane; c < n16; c += 32) acc += dot_bf16x8(__ldg(h4 + c), __ldg(d4 + c));
+    unsigned long long acc2 = 0ull;
+    for (int c = lane; c < n16; c += 32) {
+      const uint4 dv = __ldg(d4 + c);
+      const float4 ha = hf4[2 * c], hb = hf4[2 * c + 1];
+      acc2 = fma_f32x2(widen_bf16x2(dv.x), f32x2(ha.x, ha.y), acc2);
+      acc2 = fma_f32x2(widen_bf16x2(dv.y), f32x2(ha.z, ha.w), acc2);
+      acc2 = fma_f32x2(widen_bf16x2(dv.z), f32x2(hb.x, hb.y), acc2);
+      acc2 = fma_f32x2(widen_bf16x2(dv.w), f32x2(hb.z, hb.w), acc2);
+    }
+    float a0, a1;
+    f32x2_split(acc2, a0, a1);
+    float acc = a0 + a1;
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
     if (lane == 0) sm.wt[q] = acc / (1.0f + expf(-acc));   // silu
@@ -381,24 +404,24 @@ __global__ void __launch_bounds__(kRouteThreads)
   // share of the kept experts (groups of threads split the experts when the
   // row has fewer pieces than the block has threads); the groups' partial
   // sums meet in shared memory (the candidate-key buffer, free by now)
-  const int groups = n16 >= static_cast<int>(blockDim.x) ? 1 : static_cast<int>(blockDim.x) / n16;
   float* part = reinterpret_cast<float*>(sm.keys);   // [groups - 1][hidden]
   for (int c0 = 0; c0 < n16; c0 += static_cast<int>(blockDim.x) / groups) {
     const int c = c0 + static_cast<int>(threadIdx.x) % (static_cast<int>(blockDim.x) / groups);
     const int grp = static_cast<int>(threadIdx.x) / (static_cast<int>(blockDim.x) / groups);
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (c < n16 && grp < groups) {
+      unsigned long long acc2[4] = {0ull, 0ull, 0ull, 0ull};   // packed channel pairs
 #pragma unroll 4
       for (int q = grp; q < k; q += groups) {
         const uint4 u = __ldg(reinterpret_cast<const uint4*>(up_embed + static_cast<size_t>(sm.ex[q]) * hidden) + c);
         const float wq = sm.wt[q];
+        const unsigned long long w2 = f32x2(wq, wq);
         const uint32_t x[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          acc[2 * i] = fmaf(wq, __uint_as_float(x[i] << 16), acc[2 * i]);
-          acc[2 * i + 1] = fmaf(wq, __uint_as_float(x[i] & 0xFFFF0000u), acc[2 * i + 1]);
-        }
+        for (int i = 0; i < 4; ++i) acc2[i] = fma_f32x2(widen_bf16x2(x[i]), w2, acc2[i]);
       }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) f32x2_split(acc2[i], acc[2 * i], acc[2 * i + 1]);
       if (grp > 0) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) part[(grp - 1) * hidden + 8 * c + i] = acc[i];

@@ -10,9 +10,10 @@
 // w + 127 keys any of its rows keeps (or, without top-k, the kernel derives
 // the list itself: the keys up to the tile's last visible row); the kernel
 // streams those keys in tiles of 128 and never touches a key the tile does
-// not keep.  The kernel is persistent: one CTA per SM walks a snake order over
-// the work items (heaviest row tiles first), and every role counts key tiles
-// across items so rings and barrier phases carry on from item to item.
+// not keep.  The kernel is persistent: one CTA per SM walks the work items,
+// heaviest row tiles first (at d = 64 in a static snake order, at d = 128
+// drawn from a global counter), and every role counts key tiles across items
+// so rings and barrier phases carry on from item to item.
 // 384 threads in three warpgroups:
 //   * warp 0 (K producer): TMA loads the item's Q tiles (after the previous
 //     item's last Q K^T, signalled by q_empty); for every key tile it fetches

@@ -73,9 +73,7 @@ constexpr int kRegsSoftmax = 208;
 static_assert(kRegsControl % 8 == 0 && kRegsSoftmax % 8 == 0, "setmaxnreg takes multiples of 8");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
-// every kPolyEvery-th pair of probabilities in a row is computed on the FMA pipe
-// (exp2_poly_x2), the rest on the MUFU
-constexpr int kPolyEvery = 5;
+
 constexpr int kXBytes = kKeyTile * 32;       // 128 rows x 16 bf16 extra K columns (bias / ones)
 // A gathered K or V tile is 32 groups of four listed rows, one tile::gather4
 // per group and 64-column slab.  A warp issues its lanes' copies one after
@@ -110,6 +108,10 @@ struct Cfg {
   // the softmax releases S as soon as it has read it, and the next S = Q K^T
   // overlaps the current softmax.  At d = 128 (O 2x128) P is written over S.
   static constexpr bool kSepP = D == 64;
+  // every kPolyEvery-th pair of probabilities in a row is computed on the FMA
+  // pipe (exp2_poly_x2), the rest on the MUFU: measured best at 1/5 for d = 64
+  // (both heads' exponentials run at once) and 1/8 for d = 128
+  static constexpr int kPolyEvery = D == 128 ? 8 : 5;
   // d = 128 splits its gathers over a third warp (kGatherSplit); at d = 64 a
   // tile is half as many copies and the split measured slower, so the K and
   // V producers issue all of theirs
@@ -948,7 +950,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               fma_f32x2(f32x2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), scale2, nm2);
           float x0, x1, p0, p1;
           f32x2_split(x2, x0, x1);
-          if (((k >> 1) % kPolyEvery) == kPolyEvery - 1) {
+          if (((k >> 1) % C::kPolyEvery) == C::kPolyEvery - 1) {
             exp2_poly_x2(x0, x1, p0, p1);
           } else {
             p0 = fast_exp2(x0);

@@ -391,8 +391,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // atomic's latency is hidden) and publishes each number in ring slot
   // i % kItemRing; the other roles wait for the slot, read it and release it.
   // The last CTA to finish resets the counter (the workspace starts zeroed).
-  uint32_t* sched = err + 16;        // items handed out beyond the first wave
-  uint32_t* sched_done = err + 17;   // CTAs finished
+  uint32_t* sched = err + kHdrItemWord;        // items handed out beyond the first wave
+  uint32_t* sched_done = err + kHdrDoneWord;   // CTAs finished
   int* ring = reinterpret_cast<int*>(smem + C::kOffRing);
   int next_w = 0;                    // the K producer's prefetched number
   auto fetch_item = [&](int i) -> int {

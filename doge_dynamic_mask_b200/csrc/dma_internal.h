@@ -31,8 +31,13 @@ enum DeviceError : uint32_t {
   kDevErrTimeoutBase = 100,  // 100 + site: a bounded wait gave up
 };
 
-// Workspace header: status word at offset 0; the rest of the first 256 bytes is reserved.
+// Workspace header: status word at offset 0; the prefill attention's
+// work-item counter and finished-CTA counter at words kHdrItemWord and
+// kHdrDoneWord (the last CTA of each launch returns both to zero); the rest of
+// the first 256 bytes is reserved.
 constexpr size_t kHeaderBytes = 256;
+constexpr int kHdrItemWord = 16;
+constexpr int kHdrDoneWord = 17;
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

@@ -34,8 +34,10 @@
  *     fail synchronously on argument errors and launch errors.  Faults found
  *     on the device (a length outside [1, Lk], a bounded wait that gave up) are
  *     recorded in the workspace's status word; read them with dma_check().
- *   - A workspace must be zeroed once before its first use (the status word
- *     lives in its first bytes); kernels only ever set that word.
+ *   - A workspace must be zeroed once before its first use.  Its first 256
+ *     bytes are a header: the status word at byte 0 (kernels only ever set
+ *     it) and, at bytes 64-71, a work-item counter of the d = 128 prefill
+ *     attention, which every such call leaves at zero when it ends.
  *   - Calls on different streams must use different workspaces.
  */
 #ifndef DMA_H_

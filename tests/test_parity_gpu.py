@@ -211,7 +211,7 @@ def test_prefill_repeated_calls_share_a_workspace(dma, w_):
                                             workspace=ws).clone())
         assert dma.dma_check(ws) == 0
         header = ws[:256].view(torch.int32).cpu()
-        assert int(header[16]) == 0 and int(header[17]) == 0, "work-item counter not reset"
+        assert int(header[16]) == 0 and int(header[17]) == 0, "work-item counter (bytes 64-71) not reset"
     for i, o in enumerate(outs):
         assert_out_close(o, want, f"call {i}")
     if w_.w >= w_.L:

@@ -70,8 +70,17 @@ struct PrefillSelSmem {
 };
 
 // prefill selector CTA: threads, and CTAs resident per SM (64 registers a thread)
+// Two CTA shapes (threads, CTAs per SM at 64 registers a thread or fewer):
+// 512 x 2 for sequences of fewer than kSelLongRowTiles row tiles, 256 x 3
+// beyond (smaller blocks pay less at the per-tile barriers, and the longer
+// prefix selections of long sequences spread over more CTAs).  Measured: the
+// padded sparse workload (64 row tiles) 0.074 ms with 512 x 2 and 0.076 ms
+// with 256 x 3; the long one (256 row tiles) 0.108 and 0.100 ms.
 constexpr int kSelPrefillThreads = 512;
 constexpr int kSelPrefillMinBlocks = 2;
+constexpr int kSelPrefillThreadsLong = 256;
+constexpr int kSelPrefillMinBlocksLong = 3;
+constexpr int kSelLongRowTiles = 128;
 
 // at most this many consecutive row tiles per prefill-selector CTA (see
 // select_prefill_kernel); the launcher picks fewer when the grid would not
@@ -602,7 +611,8 @@ static __device__ __noinline__ void list_whole_set(const uint64_t* K, int w, int
 // key is kept up to the first row whose tau lies above it.  The list holds the
 // keys every row keeps, then the others, each class in U's (descending key)
 // order; consecutive lanes write consecutive entries.
-__global__ void __launch_bounds__(kSelPrefillThreads, kSelPrefillMinBlocks) select_prefill_kernel(const float* __restrict__ dt,
+template <int kThreads_, int kMinBlocks_>
+__global__ void __launch_bounds__(kThreads_, kMinBlocks_) select_prefill_kernel(const float* __restrict__ dt,
                                                                      const int32_t* __restrict__ lengths, int Hkv,
                                                                      int L, int w, int tpc, PrefillPlan plan,
                                                                      uint32_t* err) {
@@ -1098,24 +1108,34 @@ cudaError_t launch_select_prefill(const float* dt, const int32_t* lengths, const
   const int L = g.Lk;
   const int ucap = L > g.w ? g.w + kRowTile : 0;
   const size_t smem = select_prefill_smem_bytes(ucap);
-  cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(select_prefill_kernel), static_cast<int>(smem));
+  const bool long_rows = plan.n_row_tiles >= kSelLongRowTiles;
+  const void* kfn = long_rows
+                        ? reinterpret_cast<const void*>(select_prefill_kernel<kSelPrefillThreadsLong, kSelPrefillMinBlocksLong>)
+                        : reinterpret_cast<const void*>(select_prefill_kernel<kSelPrefillThreads, kSelPrefillMinBlocks>);
+  cudaError_t e = ensure_dyn_smem(kfn, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   // row tiles per CTA: a run's first tile selects over its prefix and sorts
   // its kept set, every later one only merges its new keys, so runs should be
   // long; the grid should still fill one wave of resident CTAs with the tiles
   // that need the top-k (rows below keep_window_size keep every visible key
   // and cost little).  Measured on the sparse and long workloads: 3 and 8
-  // tiles per CTA (this rule gives 3 and 7).
+  // tiles per CTA with 512-thread CTAs (this rule gives 3 and 7); the long
+  // workload's 256-thread CTAs get 5.
   const int nsm = sm_count();
   if (nsm <= 0) return cudaErrorInvalidDevice;
   const long long free_tiles = L > g.w ? std::min<long long>(plan.n_row_tiles, g.w / kRowTile) : plan.n_row_tiles;
   const long long topk_tiles = (static_cast<long long>(plan.n_row_tiles) - free_tiles) * g.Hkv * g.B;
-  const long long slots = static_cast<long long>(kSelPrefillMinBlocks) * nsm;
+  const long long slots =
+      static_cast<long long>(long_rows ? kSelPrefillMinBlocksLong : kSelPrefillMinBlocks) * nsm;
   long long tpc = (topk_tiles + slots - 1) / slots;
   tpc = tpc < 1 ? 1 : (tpc > kSelTilesPerCtaMax ? kSelTilesPerCtaMax : tpc);
   dim3 grid(g.Hkv, g.B, static_cast<unsigned>((plan.n_row_tiles + tpc - 1) / tpc));
-  return launch_after(select_prefill_kernel, grid, dim3(kSelPrefillThreads), smem, s, dt, lengths, g.Hkv, L, g.w,
-                      static_cast<int>(tpc), plan, err);
+  if (long_rows)
+    return launch_after(select_prefill_kernel<kSelPrefillThreadsLong, kSelPrefillMinBlocksLong>, grid,
+                        dim3(kSelPrefillThreadsLong), smem, s, dt, lengths, g.Hkv, L, g.w, static_cast<int>(tpc), plan,
+                        err);
+  return launch_after(select_prefill_kernel<kSelPrefillThreads, kSelPrefillMinBlocks>, grid, dim3(kSelPrefillThreads),
+                      smem, s, dt, lengths, g.Hkv, L, g.w, static_cast<int>(tpc), plan, err);
 }
 
 cudaError_t launch_select_decode(const float* dt, const int32_t* lengths, const Geometry& g,

@@ -12,23 +12,24 @@
 //   a_i   = pos * theta^(-2i/d),  i < d/2,  pos = positions[b] + t
 //
 // Design.  Memory-bound: every projected row is read once and written once.
-// Persistent CTAs (two per SM) walk the tokens.  A token's q, k and v rows are
-// contiguous in each tensor, so one thread brings them into a ring of shared
-// memory stages with three bulk copies per token; with the ring several
-// tokens ahead, each SM keeps about 64 KB of reads in flight, which is what
-// the HBM latency needs.  The d/2 angles of a position are formed in double
-// precision (a position of 10^5 times a frequency near 1 would lose about
-// 2^-7 rad of its angle in float32, the size of a bf16 rounding) as turns
-// (pos times theta^(-2i/d) / (2 pi), the factors formed once per call by the
-// launcher), reduced to their fractional part, and their cosines and sines
-// taken in float32 (sincospi); they are formed one token ahead, while the
-// current token's rows are processed.  Each group of d/8 threads owns one
-// head row as sixteen-byte vectors (eight bf16 channels per thread): the mean
-// square is a group shuffle reduction, and channel i's rotation partner
-// i + d/2 sits in the thread d/16 positions away, one shuffle.  A thread's
-// channels are the same for every row and token it handles, so its norm
-// weights stay in registers.  Arithmetic is float32 with one rounding to bf16
-// at the end; V rows are copied bit for bit.
+// Persistent CTAs (two per SM, 128 threads) walk contiguous chunks of tokens.
+// A token's q, k and v rows are contiguous in each tensor, so one thread
+// brings a stage of tokens into a three-stage shared-memory ring with three
+// bulk copies, and sends each token's rows out again with one bulk copy per
+// tensor once they are done; the stores read a stage while the next one is
+// processed, and a stage is refilled as soon as its stores have read it.  The
+// d/2 angles of a position are formed in double precision (a position of 10^5
+// times a frequency near 1 would lose about 2^-7 rad of its angle in float32,
+// the size of a bf16 rounding) as turns (pos times theta^(-2i/d) / (2 pi), the
+// factors formed once per call by the launcher), reduced to their fractional
+// part, and their cosines and sines taken in float32 (sincospi); they are
+// formed one stage ahead, while the current stage's rows are processed.  Each
+// thread owns whole q and k rows of the stage and rewrites them in place: one
+// pass for the mean square, one for the scaled rotation of channel pairs
+// (i, i + d/2), both reading 16-byte vectors in an order rotated by the row
+// index so that a warp's reads spread over all banks.  Arithmetic is float32
+// (packed pairs) with one rounding to bf16 at the end; V rows are copied bit
+// for bit.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -36,9 +37,9 @@
 namespace dma {
 namespace {
 
-constexpr int kPrologueThreads = 256;
-constexpr int kPrologueMaxStages = 2;
-constexpr int kPrologueMinBlocks = 2;             // CTAs per SM (128 registers a thread)
+constexpr int kPrologueThreads = 128;
+constexpr int kPrologueStages = 3;
+constexpr int kPrologueMinBlocks = 2;             // CTAs per SM
 constexpr int kPrologueMaxTokens = 16;            // tokens per stage
 constexpr int kPrologueAngles = kPrologueMaxTokens * 64 / kPrologueThreads;   // angles per thread and stage, at most
 constexpr int kPrologueStageBytes = 32 * 1024;   // rows of one ring stage (whole tokens)
@@ -62,6 +63,18 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                : "memory");
 }
 
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
+// from shared to global memory (bulk async-group completion).
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(dst)),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // theta^(-2i/d) / (2 pi) for i < d/2: each angle in turns is pos times one of
 // these, formed once per call in double precision by the launcher
 struct RopeTurns {
@@ -69,37 +82,44 @@ struct RopeTurns {
 };
 
 // One ring stage holds the rows of `nts` consecutive tokens of the CTA's
-// chunk: [q rows of those tokens][k rows][v rows], each region one bulk copy.
-// Its angles (cosines, then sines, per token and pair index) and each token's
-// cache row (-1 outside the cache) sit in one of two slots, formed while the
-// previous stage is processed.
+// chunk: [q rows of those tokens][k rows][v rows], each region one bulk copy
+// in.  Each thread normalises and rotates whole q or k rows in place (its own
+// rows, read in an order rotated by the row index so that a warp's 16-byte
+// reads spread over every bank); then one thread sends each token's q, k and
+// v rows out with a bulk copy per tensor.  A stage's angles (cosines, then
+// sines, per token and pair index) and each token's cache row (-1 outside
+// the cache) sit in one of two slots, formed while the previous stage is
+// processed.
 template <int D>
 __global__ void __launch_bounds__(kPrologueThreads, kPrologueMinBlocks)
     prologue_kernel(const unsigned char* __restrict__ q, const unsigned char* __restrict__ k,
                     const unsigned char* __restrict__ v, const float* __restrict__ q_w,
                     const float* __restrict__ k_w, float eps, const __grid_constant__ RopeTurns turns,
                     const int32_t* __restrict__ positions, int L, int Lmax, int Hq, int Hkv, int ntok, int chunk,
-                    int nts, int stages, uint4* __restrict__ q_out, uint4* __restrict__ k_cache,
-                    uint4* __restrict__ v_cache, uint32_t* err) {
-  constexpr int kLanesPerRow = D / 8;               // 16-byte vectors per head row
-  constexpr int kHalf = kLanesPerRow / 2;           // lane distance of channel i's partner i + d/2
-  static_assert(kPrologueThreads % kLanesPerRow == 0, "a thread keeps its channels");
+                    int nts, unsigned char* __restrict__ q_out, unsigned char* __restrict__ k_cache,
+                    unsigned char* __restrict__ v_cache, uint32_t* err) {
+  constexpr int kChunks = D / 8;          // 16-byte chunks (eight channels) per row
+  constexpr int kHalfC = kChunks / 2;     // chunk c pairs with chunk c + kHalfC (channel i with i + d/2)
   extern __shared__ __align__(128) unsigned char dyn[];
-  __shared__ uint64_t full[kPrologueMaxStages];
+  __shared__ uint64_t full[kPrologueStages];
+  __shared__ __align__(16) float s_w[2][D];   // q_norm and k_norm weights
 
   const uint32_t qbytes = static_cast<uint32_t>(Hq) * D * 2, kvbytes = static_cast<uint32_t>(Hkv) * D * 2;
   const size_t sbytes = static_cast<size_t>(nts) * (qbytes + 2 * kvbytes);   // one stage
-  float* ang = reinterpret_cast<float*>(dyn + static_cast<size_t>(stages) * sbytes);   // [2][nts][2][D/2]
-  int* crow_s = reinterpret_cast<int*>(ang + 2 * nts * D);                              // [2][nts]
+  float* ang = reinterpret_cast<float*>(dyn + static_cast<size_t>(kPrologueStages) * sbytes);   // [2][nts][2][D/2]
+  int* crow_s = reinterpret_cast<int*>(ang + 2 * nts * D);                                      // [2][nts]
   const int tid = threadIdx.x;
-  const int sub = tid % kLanesPerRow;               // this thread's 8 channels: [8 sub, 8 sub + 8)
   const int t_begin = static_cast<int>(blockIdx.x) * chunk;
   const int t_end = min(ntok, t_begin + chunk);
   const int nst = t_end > t_begin ? (t_end - t_begin + nts - 1) / nts : 0;   // stages of this CTA
 
   if (tid == 0) {
-    for (int s = 0; s < stages; ++s) mbar_init(full + s, 1);
+    for (int s = 0; s < kPrologueStages; ++s) mbar_init(full + s, 1);
     fence_mbar_init();
+  }
+  for (int c = tid; c < D; c += kPrologueThreads) {
+    s_w[0][c] = q_w[c];
+    s_w[1][c] = k_w[c];
   }
   __syncthreads();
   // stage i of this CTA into ring slot s (thread 0)
@@ -112,9 +132,9 @@ __global__ void __launch_bounds__(kPrologueThreads, kPrologueMinBlocks)
     bulk_load(st + n * qbytes, k + static_cast<size_t>(t0) * kvbytes, n * kvbytes, full + s);
     bulk_load(st + n * (qbytes + kvbytes), v + static_cast<size_t>(t0) * kvbytes, n * kvbytes, full + s);
   };
-  int issued = nst < stages ? nst : stages;
+  const int first = nst < kPrologueStages ? nst : kPrologueStages;
   if (tid == 0)
-    for (int i = 0; i < issued; ++i) issue(i, i);
+    for (int i = 0; i < first; ++i) issue(i, i);
 
   // angles of stage i's tokens into slot i & 1: the angle in turns
   // u = pos * theta^(-2i/d) / (2 pi) in double precision; its fractional part
@@ -166,129 +186,115 @@ __global__ void __launch_bounds__(kPrologueThreads, kPrologueMinBlocks)
   int pv[kPrologueAngles];
   pos_of(0, pv);
   angles(0, pv);
-  const bool low = sub < kHalf;                     // channels below d/2
-  const int i0 = 8 * (low ? sub : sub - kHalf);     // pair index of this thread's first channel
-  const float inv_hq = 1.0f / static_cast<float>(Hq), inv_hkv = 1.0f / static_cast<float>(Hkv);
-  // norm weights of this thread's channels and, with the rotation's sign
-  // (the low half subtracts its partner's share), of its partner's channels
-  const int psub = sub ^ kHalf;
-  const float sg = low ? -1.0f : 1.0f;
-  unsigned long long wq[4], wk[4], wpq[4], wpk[4];
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    wq[c] = f32x2(q_w[8 * sub + 2 * c], q_w[8 * sub + 2 * c + 1]);
-    wk[c] = f32x2(k_w[8 * sub + 2 * c], k_w[8 * sub + 2 * c + 1]);
-    wpq[c] = f32x2(sg * q_w[8 * psub + 2 * c], sg * q_w[8 * psub + 2 * c + 1]);
-    wpk[c] = f32x2(sg * k_w[8 * psub + 2 * c], sg * k_w[8 * psub + 2 * c + 1]);
-  }
 
   int i = 0;
   for (; i < nst; ++i) {
-    const int s = i % stages;
+    const int s = i % kPrologueStages;
     const int t0 = t_begin + i * nts;
     const int n = min(nts, t_end - t0);
     pos_of(i + 1, pv);   // the next stage's positions, used after this stage's rows
-    const bool ok = mbar_wait(full + s, static_cast<uint32_t>(i / stages) & 1u, err, kDevErrTimeoutBase + 50);
+    const bool ok = mbar_wait(full + s, static_cast<uint32_t>(i / kPrologueStages) & 1u, err, kDevErrTimeoutBase + 50);
     if (__syncthreads_or(!ok)) break;   // also publishes this stage's angles
-    const uint4* st = reinterpret_cast<const uint4*>(dyn + static_cast<size_t>(s) * sbytes);
+    unsigned char* st = dyn + static_cast<size_t>(s) * sbytes;
     const float* a = ang + (i & 1) * nts * D;
     const int* crow_t = crow_s + (i & 1) * nts;
-    const int nq = n * Hq * kLanesPerRow, nk = n * Hkv * kLanesPerRow;
-    const int npieces = nq + 2 * nk;
-    const int nsteps = (npieces + 2 * kPrologueThreads - 1) / (2 * kPrologueThreads);
-    // two pieces per thread and step, kPrologueThreads apart: their chains
-    // (load, partner shuffle, mean-square reduction, rotation, store) are
-    // independent and overlap.  The shuffles run on every thread of the warp
-    // (uniform trip count).
-    for (int k2 = 0; k2 < nsteps; ++k2) {
-      bool live[2];
-      int kind[2], j[2], head[2], token[2];
-      size_t crow[2];
-      bool in_cache[2];
-      uint4 u[2];
+    const int nqr = n * Hq, nrows = n * (Hq + Hkv);   // q rows, then k rows (v rows pass through)
+    for (int r = tid; r < nrows; r += kPrologueThreads) {
+      const bool is_q = r < nqr;
+      const int j = is_q ? r / Hq : (r - nqr) / Hkv;   // token of the stage
+      uint4* row = reinterpret_cast<uint4*>(st + static_cast<size_t>(r) * D * 2);
+      const float* w = s_w[is_q ? 0 : 1];
+      const float* cs = a + j * D;            // cos of pair index i at cs[i], sin at cs[D/2 + i]
+      // mean square of the row (chunks in an order rotated by the row index)
+      unsigned long long acc = 0ull;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int piece = (2 * k2 + h) * kPrologueThreads + tid;   // in stage order: q rows, k rows, v rows
-        live[h] = piece < npieces;
-        kind[h] = piece < nq ? 0 : (piece < nq + nk ? 1 : 2);   // q, k or v
-        const int pr = (kind[h] == 0 ? piece : (kind[h] == 1 ? piece - nq : piece - nq - nk)) / kLanesPerRow;
-        const int hh = kind[h] == 0 ? Hq : Hkv;
-        // token of the stage and head of the row: pr / hh through the float
-        // reciprocal, exact here (pr < 2^12, hh <= 2^7: the quotient is at
-        // least 1/(2 hh) from an integer, far above the rounding)
-        j[h] = live[h] ? __float2int_rz((static_cast<float>(pr) + 0.5f) * (kind[h] == 0 ? inv_hq : inv_hkv)) : 0;
-        head[h] = live[h] ? pr - j[h] * hh : 0;
-        token[h] = t0 + j[h];
-        const int cr = kind[h] == 0 ? 0 : crow_t[j[h]];
-        in_cache[h] = cr >= 0;
-        crow[h] = static_cast<size_t>(cr) * Hkv + head[h];
-        u[h] = live[h] ? st[piece] : make_uint4(0u, 0u, 0u, 0u);
-        if (live[h] && kind[h] == 2 && in_cache[h]) v_cache[crow[h] * kLanesPerRow + sub] = u[h];   // V: as is
+      for (int c = 0; c < kChunks; ++c) {
+        const uint4 u = row[(c + r) % kChunks];
+        acc = fma_f32x2(widen_bf16x2(u.x), widen_bf16x2(u.x), acc);
+        acc = fma_f32x2(widen_bf16x2(u.y), widen_bf16x2(u.y), acc);
+        acc = fma_f32x2(widen_bf16x2(u.z), widen_bf16x2(u.z), acc);
+        acc = fma_f32x2(widen_bf16x2(u.w), widen_bf16x2(u.w), acc);
       }
-      if (__all_sync(0xFFFFFFFFu, (!live[0] || kind[0] == 2) && (!live[1] || kind[1] == 2))) continue;
-      // the rotation partner's raw channels, d/16 threads away in the same row
-      uint32_t pw[2][4];
-      unsigned long long xv[2][4];
-      float ss[2];
+      float a0, a1;
+      f32x2_split(acc, a0, a1);
+      const float inv = rsqrtf((a0 + a1) * (1.0f / D) + eps);
+      const unsigned long long inv2 = f32x2(inv, inv);
+      // the rotation of channel pairs (i, i + d/2), eight pairs per step
+#pragma unroll 2
+      for (int c = 0; c < kHalfC; ++c) {
+        const int cl = (c + r) % kHalfC, ch = cl + kHalfC;
+        // at d = 64 a row is 128 bytes, so rows r and r + 4 would read the
+        // same bank positions: one of them takes the high chunk first
+        const bool swap = kHalfC < 8 && ((r / kHalfC) & 1);
+        const uint4 u0 = row[swap ? ch : cl], u1 = row[swap ? cl : ch];
+        const uint4 ul = swap ? u1 : u0, uh = swap ? u0 : u1;
+        const uint32_t xl[4] = {ul.x, ul.y, ul.z, ul.w}, xh[4] = {uh.x, uh.y, uh.z, uh.w};
+        const float4* wl4 = reinterpret_cast<const float4*>(w + 8 * cl);
+        const float4* wh4 = reinterpret_cast<const float4*>(w + 8 * ch);
+        const float4* c4 = reinterpret_cast<const float4*>(cs + 8 * cl);
+        const float4* s4 = reinterpret_cast<const float4*>(cs + D / 2 + 8 * cl);
+        const float4 wl0 = wl4[0], wl1 = wl4[1], wh0 = wh4[0], wh1 = wh4[1];
+        const float4 c0 = c4[0], c1 = c4[1], s0 = s4[0], s1 = s4[1];
+        const unsigned long long wlv[4] = {f32x2(wl0.x, wl0.y), f32x2(wl0.z, wl0.w), f32x2(wl1.x, wl1.y),
+                                           f32x2(wl1.z, wl1.w)};
+        const unsigned long long whv[4] = {f32x2(wh0.x, wh0.y), f32x2(wh0.z, wh0.w), f32x2(wh1.x, wh1.y),
+                                           f32x2(wh1.z, wh1.w)};
+        const unsigned long long cv[4] = {f32x2(c0.x, c0.y), f32x2(c0.z, c0.w), f32x2(c1.x, c1.y), f32x2(c1.z, c1.w)};
+        const unsigned long long sv[4] = {f32x2(s0.x, s0.y), f32x2(s0.z, s0.w), f32x2(s1.x, s1.y), f32x2(s1.z, s1.w)};
+        uint32_t ol[4], oh[4];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t uw[4] = {u[h].x, u[h].y, u[h].z, u[h].w};
-        unsigned long long acc = 0ull;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          pw[h][c] = __shfl_xor_sync(0xFFFFFFFFu, uw[c], kHalf);
-          xv[h][c] = widen_bf16x2(uw[c]);
-          acc = fma_f32x2(xv[h][c], xv[h][c], acc);
+        for (int e = 0; e < 4; ++e) {
+          const unsigned long long yl = mul_f32x2(mul_f32x2(widen_bf16x2(xl[e]), wlv[e]), inv2);
+          const unsigned long long yh = mul_f32x2(mul_f32x2(widen_bf16x2(xh[e]), whv[e]), inv2);
+          // out_i = y_i cos - y_{i+d/2} sin,  out_{i+d/2} = y_{i+d/2} cos + y_i sin
+          const unsigned long long lo = sub_f32x2(mul_f32x2(yl, cv[e]), mul_f32x2(yh, sv[e]));
+          const unsigned long long hi = fma_f32x2(yl, sv[e], mul_f32x2(yh, cv[e]));
+          float p0, p1;
+          f32x2_split(lo, p0, p1);
+          ol[e] = pack_bf16x2(p0, p1);
+          f32x2_split(hi, p0, p1);
+          oh[e] = pack_bf16x2(p0, p1);
         }
-        float a0, a1;
-        f32x2_split(acc, a0, a1);
-        ss[h] = a0 + a1;
+        const uint4 vl = make_uint4(ol[0], ol[1], ol[2], ol[3]), vh = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+        row[swap ? ch : cl] = swap ? vh : vl;
+        row[swap ? cl : ch] = swap ? vl : vh;
       }
-#pragma unroll
-      for (int o = kLanesPerRow / 2; o >= 1; o >>= 1) {
-        ss[0] += __shfl_xor_sync(0xFFFFFFFFu, ss[0], o);
-        ss[1] += __shfl_xor_sync(0xFFFFFFFFu, ss[1], o);
-      }
-      // out = inv (w x cos + w' x' sin): the row's norm factor, this channel's
-      // weight and the partner's signed weight
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (!live[h] || kind[h] == 2) continue;
-        const float inv = rsqrtf(ss[h] * (1.0f / D) + eps);
-        const unsigned long long inv2 = f32x2(inv, inv);
-        const float4* cp = reinterpret_cast<const float4*>(a + j[h] * D + i0);
-        const float4* sp = reinterpret_cast<const float4*>(a + j[h] * D + D / 2 + i0);
-        const float4 c0 = cp[0], c1 = cp[1], s0 = sp[0], s1 = sp[1];
-        const unsigned long long cs2[4] = {f32x2(c0.x, c0.y), f32x2(c0.z, c0.w), f32x2(c1.x, c1.y), f32x2(c1.z, c1.w)};
-        const unsigned long long sn2[4] = {f32x2(s0.x, s0.y), f32x2(s0.z, s0.w), f32x2(s1.x, s1.y), f32x2(s1.z, s1.w)};
-        const bool isq = kind[h] == 0;
-        uint32_t pk[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const unsigned long long y = mul_f32x2(xv[h][c], isq ? wq[c] : wk[c]);
-          const unsigned long long yp = mul_f32x2(widen_bf16x2(pw[h][c]), isq ? wpq[c] : wpk[c]);
-          const unsigned long long t = mul_f32x2(fma_f32x2(yp, sn2[c], mul_f32x2(y, cs2[c])), inv2);
-          float lo, hi;
-          f32x2_split(t, lo, hi);
-          pk[c] = pack_bf16x2(lo, hi);
+    }
+    fence_proxy_async_smem();   // the rows written above are read by the bulk stores
+    __syncthreads();
+    if (tid == 0) {
+      // each token's rows out: q to q_out, k and v to its cache row
+      for (int jj = 0; jj < n; ++jj) {
+        const int token = t0 + jj;
+        bulk_store(q_out + static_cast<size_t>(token) * qbytes, st + static_cast<size_t>(jj) * qbytes, qbytes);
+        const int cr = crow_t[jj];
+        if (cr >= 0) {
+          bulk_store(k_cache + static_cast<size_t>(cr) * kvbytes,
+                     st + static_cast<size_t>(n) * qbytes + static_cast<size_t>(jj) * kvbytes, kvbytes);
+          bulk_store(v_cache + static_cast<size_t>(cr) * kvbytes,
+                     st + static_cast<size_t>(n) * (qbytes + kvbytes) + static_cast<size_t>(jj) * kvbytes, kvbytes);
         }
-        const uint4 o = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        if (isq) __stcs(q_out + (static_cast<size_t>(token[h]) * Hq + head[h]) * kLanesPerRow + sub, o);
-        else if (in_cache[h]) k_cache[crow[h] * kLanesPerRow + sub] = o;
+      }
+      bulk_commit();
+      // the stage of the previous iteration is refilled once its stores have
+      // read it (this iteration's stores may still be reading)
+      if (i >= 1 && i - 1 + kPrologueStages < nst) {
+        bulk_wait_read_1();
+        fence_proxy_async_smem();
+        issue(i - 1 + kPrologueStages, (i - 1) % kPrologueStages);
       }
     }
     angles(i + 1, pv);   // the next stage's, while the others finish this one
-    __syncthreads();   // ring slot s has been read
-    if (tid == 0 && issued < nst) {
-      fence_proxy_async_smem();   // the reads above come before the copy's writes
-      issue(issued, issued % stages);
-      ++issued;
-    }
   }
-  // a wait that gave up: the copies still in flight land before the CTA exits
-  if (tid == 0)
-    for (int j = i; j < issued; ++j)
-      mbar_wait(full + j % stages, static_cast<uint32_t>(j / stages) & 1u, err, kDevErrTimeoutBase + 51);
+  if (tid == 0) {
+    bulk_wait_all();   // every store has been applied before the CTA exits
+    // a wait that gave up: the loads still in flight land first
+    // (stages 0 .. 2 at the start, then one more per finished iteration)
+    const int issued = i + kPrologueStages - 1 > kPrologueStages ? i + kPrologueStages - 1 : kPrologueStages;
+    for (int j = i; j < nst && j < issued; ++j)
+      mbar_wait(full + j % kPrologueStages, static_cast<uint32_t>(j / kPrologueStages) & 1u, err,
+                kDevErrTimeoutBase + 51);
+  }
 }
 
 }  // namespace
@@ -303,11 +309,10 @@ cudaError_t launch_prologue(const void* q, const void* k, const void* v, const f
   const double log_theta = log(static_cast<double>(theta));
   for (int i = 0; i < d / 2; ++i) turns.t[i] = exp(-2.0 * i / d * log_theta) * 0.15915494309189535;   // / (2 pi)
   const long long tbytes = static_cast<long long>(Hq + 2 * Hkv) * d * 2;   // one token's rows
-  // tokens per stage: about 32 KB of rows (at most 16 tokens), two stages
+  // tokens per stage: about 32 KB of rows (at most 16 tokens), three stages
   long long nts = kPrologueStageBytes / tbytes;
   nts = nts < 1 ? 1 : (nts > kPrologueMaxTokens ? kPrologueMaxTokens : nts);
-  const int stages = kPrologueMaxStages;
-  const long long smem = stages * nts * tbytes + 2LL * nts * d * 4 + 2LL * nts * 4;
+  const long long smem = kPrologueStages * nts * tbytes + 2LL * nts * d * 4 + 2LL * nts * 4;
   if (smem > 200 * 1024) return cudaErrorInvalidValue;
   const int nsm = sm_count();
   if (nsm <= 0) return cudaErrorInvalidDevice;
@@ -323,15 +328,15 @@ cudaError_t launch_prologue(const void* q, const void* k, const void* v, const f
   if (d == 64) {
     if ((e = ensure_dyn_smem(reinterpret_cast<const void*>(prologue_kernel<64>), static_cast<int>(smem))) != cudaSuccess) return e;
     prologue_kernel<64><<<grid, block, static_cast<size_t>(smem), s>>>(qb, kb, vb, q_w, k_w, eps, turns, positions, L, Lmax, Hq, Hkv,
-                                                  static_cast<int>(tokens), static_cast<int>(chunk), static_cast<int>(nts), stages,
-                                                  static_cast<uint4*>(q_out),
-                                                  static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), err);
+                                                  static_cast<int>(tokens), static_cast<int>(chunk), static_cast<int>(nts),
+                                                  static_cast<unsigned char*>(q_out),
+                                                  static_cast<unsigned char*>(k_cache), static_cast<unsigned char*>(v_cache), err);
   } else {
     if ((e = ensure_dyn_smem(reinterpret_cast<const void*>(prologue_kernel<128>), static_cast<int>(smem))) != cudaSuccess) return e;
     prologue_kernel<128><<<grid, block, static_cast<size_t>(smem), s>>>(qb, kb, vb, q_w, k_w, eps, turns, positions, L, Lmax, Hq, Hkv,
-                                                   static_cast<int>(tokens), static_cast<int>(chunk), static_cast<int>(nts), stages,
-                                                  static_cast<uint4*>(q_out),
-                                                   static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), err);
+                                                   static_cast<int>(tokens), static_cast<int>(chunk), static_cast<int>(nts),
+                                                  static_cast<unsigned char*>(q_out),
+                                                   static_cast<unsigned char*>(k_cache), static_cast<unsigned char*>(v_cache), err);
   }
   return cudaGetLastError();
 }

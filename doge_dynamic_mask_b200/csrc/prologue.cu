@@ -12,21 +12,22 @@
 //   a_i   = pos * theta^(-2i/d),  i < d/2,  pos = positions[b] + t
 //
 // Design.  Memory-bound: every projected row is read once and written once.
-// Persistent CTAs (two per SM, 128 threads) walk contiguous chunks of tokens.
+// Persistent CTAs (two per SM, 256 threads) walk contiguous chunks of tokens.
 // A token's q, k and v rows are contiguous in each tensor, so one thread
 // brings a stage of tokens into a three-stage shared-memory ring with three
 // bulk copies, and sends each token's rows out again with one bulk copy per
 // tensor once they are done; the stores read a stage while the next one is
-// processed, and a stage is refilled as soon as its stores have read it.  The
+// processed, and a stage is refilled once its stores have read it.  The
 // d/2 angles of a position are formed in double precision (a position of 10^5
 // times a frequency near 1 would lose about 2^-7 rad of its angle in float32,
 // the size of a bf16 rounding) as turns (pos times theta^(-2i/d) / (2 pi), the
 // factors formed once per call by the launcher), reduced to their fractional
 // part, and their cosines and sines taken in float32 (sincospi); they are
-// formed one stage ahead, while the current stage's rows are processed.  Each
-// thread owns whole q and k rows of the stage and rewrites them in place: one
-// pass for the mean square, one for the scaled rotation of channel pairs
-// (i, i + d/2), both reading 16-byte vectors in an order rotated by the row
+// formed one stage ahead, while the current stage's rows are processed.  Two
+// adjacent lanes own each q or k row of the stage and rewrite it in place,
+// each taking every other 16-byte vector: one pass for the mean square (the
+// two halves joined by one shuffle), one for the scaled rotation of channel
+// pairs (i, i + d/2), both reading the vectors in an order rotated by the row
 // index so that a warp's reads spread over all banks.  Arithmetic is float32
 // (packed pairs) with one rounding to bf16 at the end; V rows are copied bit
 // for bit.
@@ -37,8 +38,9 @@
 namespace dma {
 namespace {
 
-constexpr int kPrologueThreads = 128;
+constexpr int kPrologueThreads = 256;
 constexpr int kPrologueStages = 3;
+constexpr int kLanes = 2;                         // adjacent lanes sharing one row
 constexpr int kPrologueMinBlocks = 2;             // CTAs per SM
 constexpr int kPrologueMaxTokens = 16;            // tokens per stage
 constexpr int kPrologueAngles = kPrologueMaxTokens * 64 / kPrologueThreads;   // angles per thread and stage, at most
@@ -83,8 +85,8 @@ struct RopeTurns {
 
 // One ring stage holds the rows of `nts` consecutive tokens of the CTA's
 // chunk: [q rows of those tokens][k rows][v rows], each region one bulk copy
-// in.  Each thread normalises and rotates whole q or k rows in place (its own
-// rows, read in an order rotated by the row index so that a warp's 16-byte
+// in.  Pairs of lanes normalise and rotate the q and k rows in place (a row
+// per pair, read in an order rotated by the row index so that a warp's 16-byte
 // reads spread over every bank); then one thread sends each token's q, k and
 // v rows out with a bulk copy per tensor.  A stage's angles (cosines, then
 // sines, per token and pair index) and each token's cache row (-1 outside
@@ -199,17 +201,24 @@ __global__ void __launch_bounds__(kPrologueThreads, kPrologueMinBlocks)
     const float* a = ang + (i & 1) * nts * D;
     const int* crow_t = crow_s + (i & 1) * nts;
     const int nqr = n * Hq, nrows = n * (Hq + Hkv);   // q rows, then k rows (v rows pass through)
-    for (int r = tid; r < nrows; r += kPrologueThreads) {
+    // kLanes adjacent lanes per row: lane h takes chunks kLanes * v + h
+    const int h = tid & (kLanes - 1);
+    for (int base = 0; base < nrows; base += kPrologueThreads / kLanes) {
+      const int r = base + tid / kLanes;
+      const bool act = r < nrows;
+      const unsigned mask = __ballot_sync(0xffffffffu, act);
+      if (!act) continue;
       const bool is_q = r < nqr;
       const int j = is_q ? r / Hq : (r - nqr) / Hkv;   // token of the stage
       uint4* row = reinterpret_cast<uint4*>(st + static_cast<size_t>(r) * D * 2);
       const float* w = s_w[is_q ? 0 : 1];
       const float* cs = a + j * D;            // cos of pair index i at cs[i], sin at cs[D/2 + i]
-      // mean square of the row (chunks in an order rotated by the row index)
+      // mean square of the row: this lane's chunks 2v + h, v in an order
+      // rotated by the row index, then the partner lane's share
       unsigned long long acc = 0ull;
 #pragma unroll
-      for (int c = 0; c < kChunks; ++c) {
-        const uint4 u = row[(c + r) % kChunks];
+      for (int c = 0; c < kChunks / kLanes; ++c) {
+        const uint4 u = row[kLanes * ((c + r) % (kChunks / kLanes)) + h];
         acc = fma_f32x2(widen_bf16x2(u.x), widen_bf16x2(u.x), acc);
         acc = fma_f32x2(widen_bf16x2(u.y), widen_bf16x2(u.y), acc);
         acc = fma_f32x2(widen_bf16x2(u.z), widen_bf16x2(u.z), acc);
@@ -217,15 +226,19 @@ __global__ void __launch_bounds__(kPrologueThreads, kPrologueMinBlocks)
       }
       float a0, a1;
       f32x2_split(acc, a0, a1);
-      const float inv = rsqrtf((a0 + a1) * (1.0f / D) + eps);
+      float ss = a0 + a1;
+#pragma unroll
+      for (int o = 1; o < kLanes; o <<= 1) ss += __shfl_xor_sync(mask, ss, o);
+      const float inv = rsqrtf(ss * (1.0f / D) + eps);
       const unsigned long long inv2 = f32x2(inv, inv);
-      // the rotation of channel pairs (i, i + d/2), eight pairs per step
+      // the rotation of channel pairs (i, i + d/2), eight pairs per step:
+      // this lane's low chunks 2v + h
 #pragma unroll 2
-      for (int c = 0; c < kHalfC; ++c) {
-        const int cl = (c + r) % kHalfC, ch = cl + kHalfC;
-        // at d = 64 a row is 128 bytes, so rows r and r + 4 would read the
+      for (int c = 0; c < kHalfC / kLanes; ++c) {
+        const int cl = kLanes * ((c + r) % (kHalfC / kLanes)) + h, ch = cl + kHalfC;
+        // at d = 64 a row is 128 bytes, so rows r and r + 4 / kLanes would read the
         // same bank positions: one of them takes the high chunk first
-        const bool swap = kHalfC < 8 && ((r / kHalfC) & 1);
+        const bool swap = kHalfC < 8 && ((r / (4 / kLanes)) & 1);
         const uint4 u0 = row[swap ? ch : cl], u1 = row[swap ? cl : ch];
         const uint4 ul = swap ? u1 : u0, uh = swap ? u0 : u1;
         const uint32_t xl[4] = {ul.x, ul.y, ul.z, ul.w}, xh[4] = {uh.x, uh.y, uh.z, uh.w};

@@ -12,21 +12,23 @@
 //   a_i   = pos * theta^(-2i/d),  i < d/2,  pos = positions[b] + t
 //
 // Design.  Memory-bound: every projected row is read once and written once.
-// Persistent CTAs (two per SM, 256 threads) walk contiguous chunks of tokens.
-// A token's q, k and v rows are contiguous in each tensor, so one thread
-// brings a stage of tokens into a three-stage shared-memory ring with three
-// bulk copies, and sends each token's rows out again with one bulk copy per
-// tensor once they are done; the stores read a stage while the next one is
-// processed, and a stage is refilled once its stores have read it.  The
-// d/2 angles of a position are formed in double precision (a position of 10^5
-// times a frequency near 1 would lose about 2^-7 rad of its angle in float32,
-// the size of a bf16 rounding) as turns (pos times theta^(-2i/d) / (2 pi), the
-// factors formed once per call by the launcher), reduced to their fractional
-// part, and their cosines and sines taken in float32 (sincospi); they are
-// formed one stage ahead, while the current stage's rows are processed.  Two
-// adjacent lanes own each q or k row of the stage and rewrite it in place,
-// each taking every other 16-byte vector: one pass for the mean square (the
-// two halves joined by one shuffle), one for the scaled rotation of channel
+// Persistent CTAs (two per SM) walk contiguous chunks of tokens, with eight
+// compute warps and one copy warp each.  A token's q, k and v rows are
+// contiguous in each tensor, so the copy warp brings a stage of tokens into a
+// three-stage shared-memory ring with three bulk copies, and, once the
+// compute warps report the stage done on an mbarrier, sends each token's rows
+// out again with one bulk copy per tensor; a stage is refilled as soon as its
+// stores have read it.  The compute warps never wait for the copies: they
+// sync among themselves on a named barrier.  The d/2 angles of a position
+// are formed in double precision (a position of 10^5 times a frequency near
+// 1 would lose about 2^-7 rad of its angle in float32, the size of a bf16
+// rounding) as turns (pos times theta^(-2i/d) / (2 pi), the factors formed
+// once per call by the launcher), reduced to their fractional part, and
+// their cosines and sines taken in float32 (sincospi); they are formed one
+// stage ahead, while the current stage's rows are processed.  Two adjacent
+// lanes own each q or k row of the stage and rewrite it in place, each
+// taking every other 16-byte vector: one pass for the mean square (the two
+// halves joined by one shuffle), one for the scaled rotation of channel
 // pairs (i, i + d/2), both reading the vectors in an order rotated by the row
 // index so that a warp's reads spread over all banks.  Arithmetic is float32
 // (packed pairs) with one rounding to bf16 at the end; V rows are copied bit
@@ -38,12 +40,14 @@
 namespace dma {
 namespace {
 
-constexpr int kPrologueThreads = 256;
+constexpr int kPrologueCompute = 256;                          // warps 0-7: the rows
+constexpr int kPrologueThreads = kPrologueCompute + 32;        // warp 8: loads and stores
+constexpr int kPrologueCrowSlots = 4;                          // cache-row slots (stage % 4)
 constexpr int kPrologueStages = 3;
 constexpr int kLanes = 2;                         // adjacent lanes sharing one row
 constexpr int kPrologueMinBlocks = 2;             // CTAs per SM
 constexpr int kPrologueMaxTokens = 16;            // tokens per stage
-constexpr int kPrologueAngles = kPrologueMaxTokens * 64 / kPrologueThreads;   // angles per thread and stage, at most
+constexpr int kPrologueAngles = kPrologueMaxTokens * 64 / kPrologueCompute;   // angles per thread and stage, at most
 constexpr int kPrologueStageBytes = 32 * 1024;   // rows of one ring stage (whole tokens)
 
 __device__ __forceinline__ unsigned long long mul_f32x2(unsigned long long a, unsigned long long b) {
@@ -74,7 +78,18 @@ __device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t 
 }
 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Named barrier 1 over the kPrologueCompute compute threads; true when any of
+// them passed a true flag.
+__device__ __forceinline__ bool compute_barrier_or(bool flag) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\tbar.red.or.pred p, 1, %2, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(flag)), "n"(kPrologueCompute)
+      : "memory");
+  return r != 0;
+}
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // theta^(-2i/d) / (2 pi) for i < d/2: each angle in turns is pos times one of
@@ -85,13 +100,16 @@ struct RopeTurns {
 
 // One ring stage holds the rows of `nts` consecutive tokens of the CTA's
 // chunk: [q rows of those tokens][k rows][v rows], each region one bulk copy
-// in.  Pairs of lanes normalise and rotate the q and k rows in place (a row
-// per pair, read in an order rotated by the row index so that a warp's 16-byte
-// reads spread over every bank); then one thread sends each token's q, k and
-// v rows out with a bulk copy per tensor.  A stage's angles (cosines, then
-// sines, per token and pair index) and each token's cache row (-1 outside
-// the cache) sit in one of two slots, formed while the previous stage is
-// processed.
+// in.  Pairs of lanes of the compute warps normalise and rotate the q and k
+// rows in place (a row per pair, read in an order rotated by the row index so
+// that a warp's 16-byte reads spread over every bank); then the copy warp
+// sends each token's q, k and v rows out with a bulk copy per tensor.  A
+// stage's angles (cosines, then sines, per token and pair index) sit in one
+// of two slots and each token's cache row (-1 outside the cache) in one of
+// four, formed while the previous stage is processed; four cache-row slots
+// keep the compute warps from overwriting a stage's rows before the copy warp
+// has read them (it reads stage i's before it loads stage i + 3, and the
+// compute warps write stage i + 4's only after that load has landed).
 template <int D>
 __global__ void __launch_bounds__(kPrologueThreads, kPrologueMinBlocks)
     prologue_kernel(const unsigned char* __restrict__ q, const unsigned char* __restrict__ k,
@@ -103,20 +121,26 @@ __global__ void __launch_bounds__(kPrologueThreads, kPrologueMinBlocks)
   constexpr int kChunks = D / 8;          // 16-byte chunks (eight channels) per row
   constexpr int kHalfC = kChunks / 2;     // chunk c pairs with chunk c + kHalfC (channel i with i + d/2)
   extern __shared__ __align__(128) unsigned char dyn[];
-  __shared__ uint64_t full[kPrologueStages];
+  __shared__ uint64_t full[kPrologueStages];   // a stage's rows have landed
+  __shared__ uint64_t done[kPrologueStages];   // the compute warps have rewritten a stage's rows
+  __shared__ int abort_flag;
   __shared__ __align__(16) float s_w[2][D];   // q_norm and k_norm weights
 
   const uint32_t qbytes = static_cast<uint32_t>(Hq) * D * 2, kvbytes = static_cast<uint32_t>(Hkv) * D * 2;
   const size_t sbytes = static_cast<size_t>(nts) * (qbytes + 2 * kvbytes);   // one stage
   float* ang = reinterpret_cast<float*>(dyn + static_cast<size_t>(kPrologueStages) * sbytes);   // [2][nts][2][D/2]
-  int* crow_s = reinterpret_cast<int*>(ang + 2 * nts * D);                                      // [2][nts]
+  int* crow_s = reinterpret_cast<int*>(ang + 2 * nts * D);                  // [kPrologueCrowSlots][nts]
   const int tid = threadIdx.x;
   const int t_begin = static_cast<int>(blockIdx.x) * chunk;
   const int t_end = min(ntok, t_begin + chunk);
   const int nst = t_end > t_begin ? (t_end - t_begin + nts - 1) / nts : 0;   // stages of this CTA
 
   if (tid == 0) {
-    for (int s = 0; s < kPrologueStages; ++s) mbar_init(full + s, 1);
+    for (int s = 0; s < kPrologueStages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(done + s, kPrologueCompute / 32);
+    }
+    abort_flag = 0;
     fence_mbar_init();
   }
   for (int c = tid; c < D; c += kPrologueThreads) {
@@ -124,20 +148,76 @@ __global__ void __launch_bounds__(kPrologueThreads, kPrologueMinBlocks)
     s_w[1][c] = k_w[c];
   }
   __syncthreads();
-  // stage i of this CTA into ring slot s (thread 0)
-  auto issue = [&](int i, int s) {
-    const int t0 = t_begin + i * nts;
-    const uint32_t n = static_cast<uint32_t>(min(nts, t_end - t0));
-    unsigned char* st = dyn + static_cast<size_t>(s) * sbytes;
-    mbar_arrive_expect_tx(full + s, n * (qbytes + 2 * kvbytes));
-    bulk_load(st, q + static_cast<size_t>(t0) * qbytes, n * qbytes, full + s);
-    bulk_load(st + n * qbytes, k + static_cast<size_t>(t0) * kvbytes, n * kvbytes, full + s);
-    bulk_load(st + n * (qbytes + kvbytes), v + static_cast<size_t>(t0) * kvbytes, n * kvbytes, full + s);
-  };
-  const int first = nst < kPrologueStages ? nst : kPrologueStages;
-  if (tid == 0)
-    for (int i = 0; i < first; ++i) issue(i, i);
 
+  if (tid >= kPrologueCompute) {
+    // ===== warp 8, lane 0: loads in, stores out =====
+    if (tid != kPrologueCompute) return;
+    // stage i of this CTA into ring slot s
+    auto issue = [&](int i, int s) {
+      const int t0 = t_begin + i * nts;
+      const uint32_t n = static_cast<uint32_t>(min(nts, t_end - t0));
+      unsigned char* st = dyn + static_cast<size_t>(s) * sbytes;
+      mbar_arrive_expect_tx(full + s, n * (qbytes + 2 * kvbytes));
+      bulk_load(st, q + static_cast<size_t>(t0) * qbytes, n * qbytes, full + s);
+      bulk_load(st + n * qbytes, k + static_cast<size_t>(t0) * kvbytes, n * kvbytes, full + s);
+      bulk_load(st + n * (qbytes + kvbytes), v + static_cast<size_t>(t0) * kvbytes, n * kvbytes, full + s);
+    };
+    const int first = nst < kPrologueStages ? nst : kPrologueStages;
+    for (int i = 0; i < first; ++i) issue(i, i);
+    int issued = first;
+    for (int i = 0; i < nst; ++i) {
+      // the slot of stage i - 1 takes stage i + 2 as soon as its stores have read it
+      if (i >= 1 && issued < nst) {
+        bulk_wait_read_0();
+        fence_proxy_async_smem();
+        issue(issued, issued % kPrologueStages);
+        ++issued;
+      }
+      // stage i's rows rewritten by the compute warps (or the CTA gave up)
+      const int s = i % kPrologueStages;
+      const uint32_t par = static_cast<uint32_t>(i / kPrologueStages) & 1u;
+      bool ok = mbar_try_wait(done + s, par);
+      if (!ok) {
+        const long long t0 = clock64();
+        while (!(ok = mbar_try_wait_suspend(done + s, par, 20000u))) {
+          if (*reinterpret_cast<volatile int*>(&abort_flag)) break;
+          if (clock64() - t0 > kWaitLimitCycles) {
+            raise_error(err, kDevErrTimeoutBase + 52);
+            break;
+          }
+        }
+      }
+      if (!ok) break;
+      // each token's rows out: q to q_out, k and v to its cache row
+      const int t0 = t_begin + i * nts;
+      const int n = min(nts, t_end - t0);
+      const unsigned char* st = dyn + static_cast<size_t>(s) * sbytes;
+      const int* crow_t = crow_s + (i % kPrologueCrowSlots) * nts;
+      for (int jj = 0; jj < n; ++jj) {
+        const int token = t0 + jj;
+        bulk_store(q_out + static_cast<size_t>(token) * qbytes, st + static_cast<size_t>(jj) * qbytes, qbytes);
+        const int cr = crow_t[jj];
+        if (cr >= 0) {
+          bulk_store(k_cache + static_cast<size_t>(cr) * kvbytes,
+                     st + static_cast<size_t>(n) * qbytes + static_cast<size_t>(jj) * kvbytes, kvbytes);
+          bulk_store(v_cache + static_cast<size_t>(cr) * kvbytes,
+                     st + static_cast<size_t>(n) * (qbytes + kvbytes) + static_cast<size_t>(jj) * kvbytes, kvbytes);
+        }
+      }
+      bulk_commit();
+    }
+    bulk_wait_all();   // every store has been applied before the CTA exits
+    // the CTA gave up: loads still in flight (at most the last three issued,
+    // one per slot, so each wait's parity is unambiguous) land first
+    if (*reinterpret_cast<volatile int*>(&abort_flag)) {
+      for (int j = issued > kPrologueStages ? issued - kPrologueStages : 0; j < issued; ++j)
+        mbar_wait(full + j % kPrologueStages, static_cast<uint32_t>(j / kPrologueStages) & 1u, err,
+                  kDevErrTimeoutBase + 51);
+    }
+    return;
+  }
+
+  // ===== warps 0-7: the rows =====
   // angles of stage i's tokens into slot i & 1: the angle in turns
   // u = pos * theta^(-2i/d) / (2 pi) in double precision; its fractional part
   // r in [-1/2, 1/2] (exact in float32 to 2^-25) gives cos and sin of
@@ -151,7 +231,7 @@ __global__ void __launch_bounds__(kPrologueThreads, kPrologueMinBlocks)
     const int n = min(nts, t_end - t0);
 #pragma unroll
     for (int m = 0; m < kPrologueAngles; ++m) {
-      const int e = tid + m * kPrologueThreads;
+      const int e = tid + m * kPrologueCompute;
       if (e < n * (D / 2)) {
         const int token = t0 + e / (D / 2);
         pv[m] = positions[token / L];
@@ -165,7 +245,7 @@ __global__ void __launch_bounds__(kPrologueThreads, kPrologueMinBlocks)
     float* a = ang + (i & 1) * nts * D;
 #pragma unroll
     for (int m = 0; m < kPrologueAngles; ++m) {
-      const int e = tid + m * kPrologueThreads;
+      const int e = tid + m * kPrologueCompute;
       if (e < n * (D / 2)) {
         const int j = e / (D / 2), c = e % (D / 2);
         const int token = t0 + j;
@@ -174,7 +254,7 @@ __global__ void __launch_bounds__(kPrologueThreads, kPrologueMinBlocks)
         if (c == 0) {
           const bool in_cache = pos0 >= 0 && pos < Lmax;
           if (!in_cache) raise_error(err, kDevErrBadPosition);
-          crow_s[(i & 1) * nts + j] = in_cache ? b * Lmax + pos : -1;
+          crow_s[(i % kPrologueCrowSlots) * nts + j] = in_cache ? b * Lmax + pos : -1;
         }
         const double u = static_cast<double>(pos) * turns.t[c];
         const float r = static_cast<float>(u - rint(u));
@@ -189,21 +269,24 @@ __global__ void __launch_bounds__(kPrologueThreads, kPrologueMinBlocks)
   pos_of(0, pv);
   angles(0, pv);
 
-  int i = 0;
-  for (; i < nst; ++i) {
+  const int h = tid & (kLanes - 1);
+  for (int i = 0; i < nst; ++i) {
     const int s = i % kPrologueStages;
     const int t0 = t_begin + i * nts;
     const int n = min(nts, t_end - t0);
     pos_of(i + 1, pv);   // the next stage's positions, used after this stage's rows
     const bool ok = mbar_wait(full + s, static_cast<uint32_t>(i / kPrologueStages) & 1u, err, kDevErrTimeoutBase + 50);
-    if (__syncthreads_or(!ok)) break;   // also publishes this stage's angles
+    // the compute warps only (named barrier 1): every one has its rows, and
+    // this stage's angles (written by all of them) are visible
+    if (compute_barrier_or(!ok)) {
+      if (tid == 0) *reinterpret_cast<volatile int*>(&abort_flag) = 1;
+      break;
+    }
     unsigned char* st = dyn + static_cast<size_t>(s) * sbytes;
     const float* a = ang + (i & 1) * nts * D;
-    const int* crow_t = crow_s + (i & 1) * nts;
     const int nqr = n * Hq, nrows = n * (Hq + Hkv);   // q rows, then k rows (v rows pass through)
     // kLanes adjacent lanes per row: lane h takes chunks kLanes * v + h
-    const int h = tid & (kLanes - 1);
-    for (int base = 0; base < nrows; base += kPrologueThreads / kLanes) {
+    for (int base = 0; base < nrows; base += kPrologueCompute / kLanes) {
       const int r = base + tid / kLanes;
       const bool act = r < nrows;
       const unsigned mask = __ballot_sync(0xffffffffu, act);
@@ -274,39 +357,9 @@ __global__ void __launch_bounds__(kPrologueThreads, kPrologueMinBlocks)
       }
     }
     fence_proxy_async_smem();   // the rows written above are read by the bulk stores
-    __syncthreads();
-    if (tid == 0) {
-      // each token's rows out: q to q_out, k and v to its cache row
-      for (int jj = 0; jj < n; ++jj) {
-        const int token = t0 + jj;
-        bulk_store(q_out + static_cast<size_t>(token) * qbytes, st + static_cast<size_t>(jj) * qbytes, qbytes);
-        const int cr = crow_t[jj];
-        if (cr >= 0) {
-          bulk_store(k_cache + static_cast<size_t>(cr) * kvbytes,
-                     st + static_cast<size_t>(n) * qbytes + static_cast<size_t>(jj) * kvbytes, kvbytes);
-          bulk_store(v_cache + static_cast<size_t>(cr) * kvbytes,
-                     st + static_cast<size_t>(n) * (qbytes + kvbytes) + static_cast<size_t>(jj) * kvbytes, kvbytes);
-        }
-      }
-      bulk_commit();
-      // the stage of the previous iteration is refilled once its stores have
-      // read it (this iteration's stores may still be reading)
-      if (i >= 1 && i - 1 + kPrologueStages < nst) {
-        bulk_wait_read_1();
-        fence_proxy_async_smem();
-        issue(i - 1 + kPrologueStages, (i - 1) % kPrologueStages);
-      }
-    }
-    angles(i + 1, pv);   // the next stage's, while the others finish this one
-  }
-  if (tid == 0) {
-    bulk_wait_all();   // every store has been applied before the CTA exits
-    // a wait that gave up: the loads still in flight land first
-    // (stages 0 .. 2 at the start, then one more per finished iteration)
-    const int issued = i + kPrologueStages - 1 > kPrologueStages ? i + kPrologueStages - 1 : kPrologueStages;
-    for (int j = i; j < nst && j < issued; ++j)
-      mbar_wait(full + j % kPrologueStages, static_cast<uint32_t>(j / kPrologueStages) & 1u, err,
-                kDevErrTimeoutBase + 51);
+    __syncwarp();
+    if ((tid & 31) == 0) mbar_arrive(done + s);
+    angles(i + 1, pv);   // the next stage's, while the store warp sends this one out
   }
 }
 
@@ -325,7 +378,7 @@ cudaError_t launch_prologue(const void* q, const void* k, const void* v, const f
   // tokens per stage: about 32 KB of rows (at most 16 tokens), three stages
   long long nts = kPrologueStageBytes / tbytes;
   nts = nts < 1 ? 1 : (nts > kPrologueMaxTokens ? kPrologueMaxTokens : nts);
-  const long long smem = kPrologueStages * nts * tbytes + 2LL * nts * d * 4 + 2LL * nts * 4;
+  const long long smem = kPrologueStages * nts * tbytes + 2LL * nts * d * 4 + kPrologueCrowSlots * nts * 4LL;
   if (smem > 200 * 1024) return cudaErrorInvalidValue;
   const int nsm = sm_count();
   if (nsm <= 0) return cudaErrorInvalidDevice;

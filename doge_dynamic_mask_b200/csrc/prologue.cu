@@ -107,8 +107,8 @@ struct RopeTurns {
 // stage's angles (cosines, then sines, per token and pair index) sit in one
 // of two slots and each token's cache row (-1 outside the cache) in one of
 // four, formed while the previous stage is processed; four cache-row slots
-// keep the compute warps from overwriting a stage's rows before the copy warp
-// has read them (it reads stage i's before it loads stage i + 3, and the
+// keep the compute warps from overwriting a stage's cache-row entries before
+// the copy warp has read them (it reads stage i's before it loads stage i + 3, and the
 // compute warps write stage i + 4's only after that load has landed).
 template <int D>
 __global__ void __launch_bounds__(kPrologueThreads, kPrologueMinBlocks)

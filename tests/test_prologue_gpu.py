@@ -56,6 +56,11 @@ def run_case(dma, B, L, Lmax, Hq, Hkv, d, theta, seed, positions=None):
     (1, 5, 70000, 4, 1, 128, 500000.0),        # positions near 2^16: angles need double precision
     (4, 1, 33, 12, 4, 64, 10000.0),            # one new token per sequence (a decode step)
     (2, 17, 17, 2, 2, 64, 1000.0),             # the whole cache written
+    # several ring stages per CTA with a ragged last stage (the stage ring
+    # wraps, the copy warp refills slots, cache rows cycle through their slots)
+    (2, 3000, 3100, 8, 4, 64, 10000.0),        # 16-token stages, two per CTA
+    (1, 20000, 20000, 2, 2, 64, 10000.0),      # 16-token stages, five per CTA
+    (1, 12000, 12500, 4, 2, 128, 10000.0),     # 115 KB of shared memory: one CTA per SM
 ])
 def test_prologue_matches_oracle(dma, B, L, Lmax, Hq, Hkv, d, theta):
     positions = None if Lmax != 70000 else [Lmax - L]
